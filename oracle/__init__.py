@@ -1,0 +1,140 @@
+"""CPU oracle for silu_dot_fwd_bwd_quant_fuse -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it and never falls back to it.
+
+The arithmetic lives in ``sdq_oracle.cpp`` (plain single-threaded C++, fp64);
+this module only compiles it with g++ and marshals numpy arrays through
+ctypes.  Every function's pin is listed in the C++ file's header.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sdq_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+# No fast-math and no FMA contraction: every fp64/fp32 operation rounds once,
+# in the order written.
+CXXFLAGS = ["-O2", "-std=c++17", "-fPIC", "-shared", "-fno-fast-math",
+            "-ffp-contract=off", "-fno-strict-aliasing"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (g++; a second or two)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["g++", *CXXFLAGS, _SRC, "-o", tmp], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib() -> ctypes.CDLL:
+    """The compiled oracle.  ``SDQ_ORACLE_LIB`` names another build of the same
+    source (the mutation test plants mistakes in copies and points here)."""
+    global _lib
+    if _lib is None:
+        path = os.environ.get("SDQ_ORACLE_LIB") or build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        dbl = ctypes.c_double
+        L.oracle_bf16_rne.argtypes = [dbl]
+        L.oracle_bf16_rne.restype = ctypes.c_uint16
+        for f in (L.oracle_sigmoid, L.oracle_silu, L.oracle_silu_grad):
+            f.argtypes = [dbl]
+            f.restype = dbl
+        L.oracle_swiglu_bwd_fp64.argtypes = [dbl, dbl, dbl, P, P, P]
+        L.oracle_swiglu_bwd_fp64.restype = None
+        L.oracle_quant_group.argtypes = [P, i64, i64, P, i64, P]
+        L.oracle_quant_group.restype = None
+        L.oracle_swiglu_bwd_bf16.argtypes = [P, P, i64, i64, P, P, P]
+        L.oracle_swiglu_bwd_bf16.restype = None
+        L.oracle_silu_dot_fwd_bwd_quant_fuse.argtypes = [P, P, P, P, P, P, i64, i64, i64]
+        L.oracle_silu_dot_fwd_bwd_quant_fuse.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> ctypes.c_void_p:
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def bf16_rne(v: float) -> int:
+    """Nearest bf16 bit pattern of a double, ties to even."""
+    return int(lib().oracle_bf16_rne(float(v)))
+
+
+def sigmoid(g: float) -> float:
+    return float(lib().oracle_sigmoid(float(g)))
+
+
+def silu(g: float) -> float:
+    return float(lib().oracle_silu(float(g)))
+
+
+def silu_grad(g: float) -> float:
+    return float(lib().oracle_silu_grad(float(g)))
+
+
+def swiglu_bwd_fp64(g: float, u: float, dy: float) -> Tuple[float, float, float]:
+    """(y, d_gate, d_up) of one element in fp64, before rounding."""
+    out = [ctypes.c_double() for _ in range(3)]
+    lib().oracle_swiglu_bwd_fp64(float(g), float(u), float(dy),
+                                 *(ctypes.byref(o) for o in out))
+    return tuple(o.value for o in out)  # type: ignore[return-value]
+
+
+def quant_group(v_bf16: np.ndarray) -> Tuple[np.ndarray, float]:
+    """Quantize one group of bf16 bit patterns -> (int8 q, fp32 scale)."""
+    v = np.ascontiguousarray(v_bf16, dtype=np.uint16)
+    q = np.zeros(v.size, dtype=np.int8)
+    s = np.zeros(1, dtype=np.float32)
+    lib().oracle_quant_group(_ptr(v), v.size, 1, _ptr(q), 1, _ptr(s))
+    return q, float(s[0])
+
+
+def swiglu_bwd_bf16(x: np.ndarray, grad_y: np.ndarray):
+    """First stage: bf16 bit arrays (y, d_gate, d_up), each [M, K]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    gy = np.ascontiguousarray(grad_y, dtype=np.uint16)
+    M, K = gy.shape
+    assert x.shape == (M, 2 * K)
+    y = np.empty((M, K), np.uint16)
+    dg = np.empty((M, K), np.uint16)
+    du = np.empty((M, K), np.uint16)
+    lib().oracle_swiglu_bwd_bf16(_ptr(x), _ptr(gy), M, K, _ptr(y), _ptr(dg), _ptr(du))
+    return y, dg, du
+
+
+def silu_dot_fwd_bwd_quant_fuse(x: np.ndarray, grad_y: np.ndarray, group_size: int = 128):
+    """The whole op on uint16 (bf16 bit) arrays.
+
+    Returns ``(grad_input_q [M,2K] int8, grad_input_s [M,2K/G] f32,
+    y_q_t [K,M] int8, y_s_t [K,ceil(M/G)] f32)``.
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    gy = np.ascontiguousarray(grad_y, dtype=np.uint16)
+    M, K = gy.shape
+    assert x.shape == (M, 2 * K), (x.shape, gy.shape)
+    G = int(group_size)
+    if G < 1 or K % G:
+        raise ValueError(f"K={K} is not a multiple of group_size={G}")
+    Kg, Mg = K // G, (M + G - 1) // G
+    giq = np.zeros((M, 2 * K), np.int8)
+    gis = np.zeros((M, 2 * Kg), np.float32)
+    yqt = np.zeros((K, M), np.int8)
+    yst = np.zeros((K, Mg), np.float32)
+    rc = lib().oracle_silu_dot_fwd_bwd_quant_fuse(_ptr(x), _ptr(gy), _ptr(giq), _ptr(gis),
+                                                  _ptr(yqt), _ptr(yst), M, K, G)
+    if rc != 0:
+        raise ValueError(f"oracle rejected M={M} K={K} group_size={G}")
+    return giq, gis, yqt, yst

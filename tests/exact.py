@@ -1,0 +1,82 @@
+"""Exact-arithmetic helpers for pinning the oracle (test-only, no oracle code).
+
+These restate nothing from the oracle: bf16 rounding here is done either by
+exhaustive comparison of neighbouring bf16 values with exact rationals
+(``fractions.Fraction``) or by integer manipulation of the float64 bit
+pattern, and the second is itself checked against the first.
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+
+
+def bf16_value(bits: int) -> Fraction:
+    """Exact value of a finite bf16 bit pattern."""
+    f = np.array([bits << 16], dtype=np.uint32).view(np.float32)[0]
+    return Fraction(float(f))
+
+
+def bf16_round_bruteforce(v: float) -> int:
+    """Nearest bf16 to the double ``v`` (ties to the even pattern), found by
+    comparing the exact distance to every bf16 pattern near ``v``."""
+    if v == 0.0:
+        return 0x8000 if np.signbit(v) else 0
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    if a >= 2.0 ** 128:
+        return sign | 0x7F80
+    # A start point within a couple of patterns of the answer.
+    with np.errstate(over="ignore"):
+        f32 = np.float32(a)
+    b0 = min(0x7F7F, int(np.array([f32], dtype=np.float32).view(np.uint32)[0]) >> 16)
+    target = Fraction(a)
+    best = None
+    for b in range(max(0, b0 - 3), min(0x7F7F, b0 + 3) + 1):
+        d = abs(bf16_value(b) - target)
+        key = (d, b & 1)  # nearer first; on a tie the even pattern
+        if best is None or key < best[0]:
+            best = (key, b)
+    b = best[1]
+    # Above the largest finite value: rounds to inf when at least half an ulp past it.
+    top = bf16_value(0x7F7F)
+    if target > top and target - top >= Fraction(2) ** 119:
+        return sign | 0x7F80
+    return sign | b
+
+
+def bf16_round_bits64(v: np.ndarray) -> np.ndarray:
+    """Vectorised nearest-even rounding of float64 to bf16 bits, from the
+    float64 bit pattern (normal bf16 range and zero only; checked against
+    ``bf16_round_bruteforce`` in the tests)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    b = v.view(np.uint64)
+    sign = ((b >> np.uint64(63)) & np.uint64(1)).astype(np.uint32) << np.uint32(15)
+    exp = ((b >> np.uint64(52)) & np.uint64(0x7FF)).astype(np.int64) - 1023
+    mant = b & np.uint64((1 << 52) - 1)
+    kept = (mant >> np.uint64(45)).astype(np.int64)
+    rem = mant & np.uint64((1 << 45) - 1)
+    half = np.uint64(1 << 44)
+    up = (rem > half) | ((rem == half) & ((kept & 1) == 1))
+    body = ((exp + 127) << 7) + kept + up.astype(np.int64)
+    body = np.where(exp + 127 >= 255, 0x7F80, body)
+    zero = (b & np.uint64((1 << 63) - 1)) == 0
+    if np.any(~zero & (exp < -126)):
+        raise ValueError("subnormal bf16 results are outside this helper's range")
+    body = np.where(zero, 0, body)
+    return (sign | body.astype(np.uint32)).astype(np.uint16)
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(vals) -> np.ndarray:
+    """Exact-valued doubles (already bf16-representable) -> bf16 bits."""
+    f = np.asarray(vals, dtype=np.float64).astype(np.float32)
+    assert np.all(f.astype(np.float64) == np.asarray(vals, dtype=np.float64))
+    bits = f.view(np.uint32)
+    assert np.all((bits & np.uint32(0xFFFF)) == 0), "value is not a bf16"
+    return (bits >> np.uint32(16)).astype(np.uint16)

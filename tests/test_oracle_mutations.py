@@ -1,0 +1,62 @@
+"""The pins catch plausible mistakes: each case plants one slip in a copy of
+the oracle's source (on the CPU, in a temporary directory), builds it, and
+checks that the named pin test fails against that build."""
+from __future__ import annotations
+
+import concurrent.futures
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = [
+    ("s * (1.0 + g * (1.0 - s))", "s * (1.0 + g * (1.0 + s))", "test_silu_grad_matches_finite_difference"),
+    ("s * (1.0 + g * (1.0 - s))", "s * (1.0 + (1.0 - s))", "test_silu_grad_matches_finite_difference"),
+    ("*d_gate = dy * u * oracle_silu_grad(g);", "*d_gate = dy * oracle_silu_grad(g);", "test_swiglu_bwd_fp64_finite_differences"),
+    ("*d_up = dy * silu;", "*d_up = dy * u;", "test_swiglu_bwd_fp64_matches_torch_autograd"),
+    ("x[m * 2 * K + k]);", "x[m * 2 * K + K + k]);", "test_whole_op_gate32_closed_form"),
+    ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;", "test_quant_scale_is_amax_over_127_rounded_once"),
+    ("float r = std::nearbyint(t);", "float r = std::round(t);", "test_quant_ties_to_even_and_symmetry"),
+    ("(j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G]",
+     "(j < Kg) ? &du[m * K + j * G] : &dg[m * K + (j - Kg) * G]", "test_whole_op_gate32_closed_form"),
+    ("&y_q_t[k * M + t0], 1,", "&y_q_t[t0 * K + k], K,", "test_whole_op_gate32_closed_form"),
+    ("&y_s_t[k * Mg + i]", "&y_s_t[i * K + k]", "test_whole_op_gate32_closed_form"),
+    ("&grad_input_s[m * 2 * Kg + j]", "&grad_input_s[j * M + m]", "test_whole_op_groups_relate_to_stage1"),
+    ("const double r = std::nearbyint(a / ulp) * ulp;", "const double r = std::trunc(a / ulp) * ulp;",
+     "test_bf16_rne_bruteforce_exact_rationals"),
+    ("*scale = 1.0f;", "*scale = 0.0f;", "test_quant_zero_and_constant_groups"),
+    ("if (e < -126) e = -126;", "", "test_bf16_rne_against_torch_float32_conversion"),
+    ("return 1.0 / (1.0 + std::exp(-g));", "return 1.0 / (1.0 + std::exp(-(float)g));",
+     "test_sigmoid_matches_library_expit"),
+]
+
+
+def _run_mutant(tmp_dir, idx, old, new, pin):
+    src = open(oracle._SRC).read()
+    if src.count(old) < 1:
+        return f"mutation #{idx} no longer applies: {old!r}"
+    mutated = os.path.join(tmp_dir, f"mut{idx}.cpp")
+    with open(mutated, "w") as f:
+        f.write(src.replace(old, new, 1))
+    so = os.path.join(tmp_dir, f"libmut{idx}.so")
+    subprocess.run(["g++", *oracle.CXXFLAGS, mutated, "-o", so], check=True)
+    env = dict(os.environ, SDQ_ORACLE_LIB=so)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", pin],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    if r.returncode == 0:
+        return f"planted mistake #{idx} survived {pin}: {old!r} -> {new!r}"
+    return None
+
+
+def test_pins_catch_planted_mistakes(tmp_path):
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(2, os.cpu_count() or 2)) as ex:
+        futs = [ex.submit(_run_mutant, str(tmp_path), i, *m) for i, m in enumerate(MUTATIONS)]
+        problems = [f.result() for f in futs]
+    problems = [p for p in problems if p]
+    assert not problems, "\n".join(problems)
