@@ -1,0 +1,463 @@
+#!/usr/bin/env python3
+"""Benchmark of silu_dot_fwd_bwd_quant_fuse on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdq|reference]
+                    [--workload NAME|INDEX] [--all-workloads] [--no-cpu-baseline]
+
+One step = one call of the fused op over one synthetic batch of the
+workload (default: M=4096 tokens, K=1408 channels, the MoE-expert-sized FFN).
+Prints ONE JSON line on rank 0.
+
+Timing: W eager warm-up calls, then EXACTLY K calls replayed from CUDA
+graphs, bracketed by a barrier and a device synchronize and timed with CUDA
+events on the launching stream; the maximum over ranks is taken.  Between
+consecutive calls the inputs and outputs rotate through enough buffer sets to
+exceed 3x the L2 cache, so no call finds its data in L2.
+
+value = algorithmic bytes of all ranks / time (GB/s); the algorithmic bytes
+are 6 B read + 3 B written per (token, channel) plus the fp32 scales.
+e2e   = the same metric through the host-buffer entry point (sdq_fuse_host):
+        pinned host inputs -> device -> kernel -> all four outputs back to
+        pinned host memory, every step inside the timed region.
+cpu_baseline / --impl reference = the CPU oracle (single thread) timed on
+        bounded samples of the same workload.
+
+Multi-GPU (torchrun): each rank runs an independent replica of the workload
+(the op has no exchange step; weak scaling); NCCL carries only the barrier
+and the max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = W.WORKLOADS[1].name
+METRIC = "µs/call and achieved HBM GB/s (fraction of B200 roofline) per (M,K)"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["swiglu_backward_int8_b200/csrc/sdq_kernel.cuh",
+                  "swiglu_backward_int8_b200/csrc/sdq_ptx.cuh",
+                  "swiglu_backward_int8_b200/csrc/sdq_api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["sdq", "reference"], default="sdq")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="also time every workload and add a per_workload list")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0 = min(steps, 50)")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if a.steps < 1:
+        ap.error("--steps must be at least 1")
+    return a
+
+
+def pick_workload(name: str) -> W.Workload:
+    if name.isdigit():
+        return W.WORKLOADS[int(name)]
+    return W.BY_NAME[name]
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_sha()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload and parts[1] == sha:
+            return int(parts[2]) + int(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of this GPU's clocks and reasons."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu_uuid],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                self.samples.append({
+                    "t": time.time(), "sm": float(parts[1]), "max": float(parts[2]),
+                    "active": parts[4], "hw_slowdown": parts[5] == "Active",
+                    "hw_thermal_slowdown": parts[6] == "Active",
+                    "sw_thermal_slowdown": parts[7] == "Active",
+                    "sw_power_cap": parts[8] == "Active"})
+            except ValueError:
+                continue
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        inside = [s for s in self.samples if t0 <= s["t"] <= t1]
+        window = "timed region"
+        if not inside:  # region shorter than the sampling period: nearest samples
+            inside = [s for s in self.samples if t0 - 0.5 <= s["t"] <= t1 + 0.5] or self.samples[-3:]
+            window = "within 0.5 s of the timed region"
+        reasons = set()
+        for s in inside:
+            for k in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"):
+                if s[k]:
+                    reasons.add(k)
+        return {"sm_mhz": statistics.median(s["sm"] for s in inside),
+                "sm_max_mhz": max(s["max"] for s in inside), "reasons": sorted(reasons),
+                "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def dist_init(world, rank, local, backend="nccl"):
+    import torch
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=120),
+                                **({"device_id": torch.device("cuda", local)} if backend == "nccl" else {}))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is None:
+        return
+    import torch
+    t = torch.zeros(1, device=device)
+    dist.all_reduce(t)
+    torch.cuda.synchronize(device)
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def time_oracle(w: W.Workload, x, gy, min_seconds=10.0, max_rows=None):
+    """Time the CPU oracle (single thread) on a bounded sample of the
+    workload: its first R token rows, repeated until min_seconds pass."""
+    import oracle
+    rows = w.M if max_rows is None else min(w.M, max_rows)
+    xs, gys = x[:rows], gy[:rows]
+    sw = W.Workload(w.name + "_sample", rows, w.K, w.sigma_x, w.sigma_grad_y, w.seed)
+    oracle.silu_dot_fwd_bwd_quant_fuse(xs[:1], gys[:1])  # build/load outside the clock
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.silu_dot_fwd_bwd_quant_fuse(xs, gys)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    gbs = sw.algorithmic_bytes() * reps / el / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {w.M} token rows x K={w.K}, {reps} repetitions "
+                      f"in {el:.1f} s (single-threaded C++ oracle, fp64)"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as it stands, on host cores, each step a
+    bounded sample (one 128-token group x all K channels, cycling through the
+    workload)."""
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    w = pick_workload(args.workload)
+    x, gy = W.make_inputs(w)
+    import oracle
+    G = w.group_size
+    Mg = w.Mg
+
+    def step(s):
+        i = s % Mg
+        r0, r1 = i * G, min(w.M, i * G + G)
+        oracle.silu_dot_fwd_bwd_quant_fuse(x[r0:r1], gy[r0:r1], G)
+        return W.Workload("s", r1 - r0, w.K, 1, 1, 0).algorithmic_bytes()
+
+    for s in range(args.warmup):
+        step(s)
+    total, t0 = 0, time.perf_counter()
+    for s in range(args.steps):
+        total += step(args.warmup + s)
+    el = time.perf_counter() - t0
+    gbs = total / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "group_size": G,
+                   "step": "one 128-token group x all K channels (bounded sample)"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} steps of one 128-token group x K={w.K}"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU timing
+
+def _to_device_bf16(a_u16, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, dist):
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    M, K = w.M, w.K
+    footprint = w.algorithmic_bytes()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, -(-3 * l2 // footprint))
+    x0, g0 = _to_device_bf16(x_np, device), _to_device_bf16(gy_np, device)
+    sets = []
+    for s in range(nsets):
+        xs = x0 if s == 0 else x0.clone()
+        gs = g0 if s == 0 else g0.clone()
+        sets.append((xs, gs, sdq.allocate_outputs(M, K, device)))
+    stream = torch.cuda.current_stream(device)
+
+    def call(k):
+        xs, gs, outs = sets[k % nsets]
+        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs)
+
+    for k in range(warmup):
+        call(k)
+    torch.cuda.synchronize(device)
+    # Capture the K timed calls into CUDA graphs (chunks of at most 1000 calls).
+    chunk = min(steps, 1000)
+    graphs = []
+    done = 0
+    while done < steps:
+        n = min(chunk, steps - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+            for k in range(n):
+                call(warmup + done + k)
+        graphs.append(g)
+        done += n
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    ev0.record(stream)
+    for g in graphs:
+        g.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    barrier(dist, device)
+    ms = ev0.elapsed_time(ev1)
+    st = sdq.sdq_device_status(stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError(f"device status {sdq.status_string(st)}")
+    del graphs
+    return ms, (t0, t1), nsets
+
+
+def measure_e2e(w: W.Workload, x_np, gy_np, steps: int, device):
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    M, K = w.M, w.K
+    xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    gyh = torch.from_numpy(gy_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    outs = [t.pin_memory() for t in sdq.allocate_outputs(M, K, "cpu")]
+    ws = torch.empty(sdq.sdq_fuse_host_workspace_bytes(M, K, 0), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(3):
+        sdq.silu_dot_fwd_bwd_quant_fuse_host(xh, gyh, *outs, workspace=ws, synchronize=False)
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        sdq.silu_dot_fwd_bwd_quant_fuse_host(xh, gyh, *outs, workspace=ws, synchronize=False)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = ev0.elapsed_time(ev1) / steps
+    h2d = xh.numel() * 2 + gyh.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    return {"value": w.algorithmic_bytes() / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": steps, "path": "sdq_fuse_host (C ABI, pinned host buffers, chunked "
+                                    "H2D/kernel/D2H overlap)"}
+
+
+def run_sdq(args):
+    world, rank, local = dist_setup(args)
+    import torch
+    dist = dist_init(world, rank, local)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import swiglu_backward_int8_b200 as sdq  # fails loudly if the CUDA library is missing
+
+    w = pick_workload(args.workload)
+    # Each rank its own replica (seed offset by rank): weak scaling, no exchange.
+    wr = W.Workload(w.name, w.M, w.K, w.sigma_x, w.sigma_grad_y, w.seed + 1000 * rank,
+                    w.group_size, w.outlier_frac, w.outlier_mult, w.zero_group_every)
+    x_np, gy_np = W.make_inputs(wr)
+    peak, peak_kind = measured_peaks()
+
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    time.sleep(0.3)
+    ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, dist)
+    clocks = sampler.summary(t0, t1)
+    sampler.stop()
+    ms_max = max_over_ranks(ms, dist, device)
+    per_step_ms = ms_max / args.steps
+    bytes_step = w.algorithmic_bytes()
+    value = world * bytes_step * args.steps / (ms_max * 1e-3) / 1e9
+    achieved = bytes_step / (per_step_ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = args.e2e_steps or min(args.steps, 50)
+        e = measure_e2e(wr, x_np, gy_np, e2e_steps, device)
+        e_ms = max_over_ranks(e["ms_per_step"], dist, device)
+        e["value"] = world * bytes_step / (e_ms * 1e-3) / 1e9
+        e2e = e
+
+    per = None
+    if args.all_workloads:
+        per = []
+        for ow in W.WORKLOADS:
+            ox, og = W.make_inputs(ow)
+            osteps = max(20, min(args.steps, int(2e9 // max(1, ow.algorithmic_bytes())) + 20))
+            oms, _, ons = measure_device(ow, ox, og, osteps, args.warmup, device, dist)
+            oms = max_over_ranks(oms, dist, device)
+            us = oms / osteps * 1e3
+            gbs = ow.algorithmic_bytes() / (us * 1e-6) / 1e9
+            per.append({"workload": ow.name, "M": ow.M, "K": ow.K, "us_per_call": us,
+                        "GB_s": gbs, "frac_of_measured_hbm": gbs / peak, "frac_of_8TBs": gbs / 8000,
+                        "steps": osteps, "buffer_sets": ons})
+            del ox, og
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0)
+
+    if rank == 0:
+        traffic = recorded_traffic(w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
+            "us_per_call": per_step_ms * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "M": w.M, "K": w.K, "group_size": w.group_size,
+                       "io": "bf16 x, grad_y in; int8 + fp32 scales out",
+                       "parallelism": f"replicas x{world} (no exchange)",
+                       "l2": f"inputs+outputs rotate over {nsets} buffer sets (>= 3x L2)",
+                       "timing": "K calls replayed from CUDA graphs, CUDA events"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": traffic, "algorithmic_bytes_per_launch": bytes_step,
+                         "kernel": "sdq::fuse_kernel"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+            "kernel_sources_sha": kernel_sha(),
+        }
+        if per is not None:
+            line["per_workload"] = per
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        barrier(dist, device)
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_sdq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * sdq.h -- C ABI of the B200 (sm_100a) implementation of
+ * silu_dot_fwd_bwd_quant_fuse: fused SwiGLU forward recompute, backward, and
+ * dual-axis INT8 quantization.
+ *
+ * Source of the operation: "kernelgen-challenge-9-task3-silu-quant"
+ *   - entry point section: silu_dot_fwd_bwd_quant_fuse(x, grad_y,
+ *     grad_input_q, grad_input_s, y_q_t, y_s_t, group_size=128), outputs
+ *     preallocated by the caller and written in place;
+ *   - outputs section: recompute y = silu(gate) * up, compute the backward
+ *     gradients, write [d_gate, d_up] quantized row-wise in 128-channel groups
+ *     (grad_input_q / grad_input_s) and y transposed and quantized in
+ *     128-token groups (y_q_t / y_s_t);
+ *   - constraints list: 128x128 tiles (both quantization axes use groups of
+ *     128); forward, backward and both quantizations fused; the bf16
+ *     round-trip kept before quantization; quantization by multiplication
+ *     with a precomputed inverse scale.
+ *
+ * Definitions used (where the page is silent):
+ *   x = [gate | up] along channels, bf16 [M, 2K] row-major;
+ *   grad_y bf16 [M, K] row-major;
+ *   y = silu(g) * u, d_gate = grad_y * u * silu'(g), d_up = grad_y * silu(g),
+ *   each computed in fp32 and rounded once to bf16 (nearest even);
+ *   per group: amax = max |v|; all-zero group -> scale 1, q 0; otherwise
+ *   scale = amax / 127 (fp32, correctly rounded) and
+ *   q = round-half-even(v * (1/scale)) in [-127, 127];
+ *   a tail token group (M % 128 != 0) is quantized over the tokens it holds.
+ *
+ * Output layouts (all row-major, contiguous):
+ *   grad_input_q int8 [M, 2K]             columns 0..K-1 = d_gate, K..2K-1 = d_up
+ *   grad_input_s fp32 [M, 2K/128]         column j < K/128: d_gate group j;
+ *                                         column K/128 + j: d_up group j
+ *   y_q_t        int8 [K, M]              y transposed: y_q_t[k, m] quantizes y[m, k]
+ *   y_s_t        fp32 [K, ceil(M/128)]    y_s_t[k, i]: scale of tokens 128i..128i+127
+ *
+ * Threading and ownership: the caller owns every buffer.  The device entry
+ * point allocates nothing, keeps no pointer after it returns, and is
+ * asynchronous on the given stream (no implicit synchronization).  Calls on
+ * different streams may run concurrently; concurrent calls must not share
+ * output buffers.  Inputs and outputs must not overlap.
+ *
+ * Errors: every entry point returns an sdq_status.  On a validation error
+ * nothing is launched and nothing is written.  SDQ_ERR_CUDA means a CUDA
+ * call failed; sdq_last_cuda_error() returns its cudaError_t code.
+ */
+#ifndef SDQ_H_
+#define SDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sdq_status {
+  SDQ_OK = 0,
+  SDQ_ERR_NULL = 1,      /* a required pointer is NULL (with M > 0)                  */
+  SDQ_ERR_GROUP = 2,     /* group_size != 128                                        */
+  SDQ_ERR_SHAPE = 3,     /* M < 0, K < 1, K % 128 != 0, or a size above the limits   */
+  SDQ_ERR_ALIGN = 4,     /* x, grad_y, grad_input_q, y_q_t not 16-byte aligned, or a
+                            scale pointer not 4-byte aligned                          */
+  SDQ_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed (see sdq_last_cuda_error) */
+  SDQ_ERR_TIMEOUT = 6,   /* a device-side wait hit its time limit (sdq_device_status) */
+  SDQ_ERR_WORKSPACE = 7  /* the workspace given to sdq_fuse_host is too small        */
+} sdq_status;
+
+/* Largest accepted sizes: M < 2^31 (tensor-map coordinates are 32-bit) and
+ * K <= 2^20 channels. */
+#define SDQ_GROUP_SIZE 128
+#define SDQ_MAX_M 2147483647LL
+#define SDQ_MAX_K 1048576LL
+
+/*
+ * sdq_fuse -- the op on device buffers.
+ *   x             device, bf16 [M, 2K], 16-byte aligned
+ *   grad_y        device, bf16 [M, K], 16-byte aligned
+ *   grad_input_q  device, int8 [M, 2K], 16-byte aligned      (written)
+ *   grad_input_s  device, fp32 [M, 2K/128], 4-byte aligned   (written)
+ *   y_q_t         device, int8 [K, M], 16-byte aligned       (written)
+ *   y_s_t         device, fp32 [K, ceil(M/128)], 4-byte aligned (written)
+ *   M             tokens (rows of x), 0 <= M <= SDQ_MAX_M; M == 0 is a no-op
+ *   K             channels of gate/up, a positive multiple of 128, <= SDQ_MAX_K
+ *   group_size    must be 128
+ *   stream        a cudaStream_t (NULL = the legacy default stream)
+ * Launches one persistent kernel on the current device.  Returns SDQ_OK once
+ * the launch is enqueued.
+ */
+int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q,
+             float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M,
+             int64_t K, int32_t group_size, void* stream);
+
+/*
+ * sdq_validate -- the argument checks of sdq_fuse alone: no CUDA call, no
+ * launch.  Returns the status sdq_fuse would return before launching.
+ */
+int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
+                 const float* grad_input_s, const int8_t* y_q_t,
+                 const float* y_s_t, int64_t M, int64_t K, int32_t group_size);
+
+/*
+ * sdq_fuse_host -- the op on HOST buffers (same shapes and layouts as
+ * sdq_fuse; page-locked host memory gives overlapped copies, pageable memory
+ * works but copies synchronously).  The rows are processed in chunks through
+ * a caller-provided device workspace: host->device copy of a chunk of x and
+ * grad_y, the kernel, device->host copy of the chunk's four outputs, with the
+ * copies of one chunk overlapping the kernel of another.  Enqueued on
+ * `stream`; the host outputs are complete once `stream` has been
+ * synchronized.
+ *   workspace        device memory, 256-byte aligned, owned by the caller
+ *   workspace_bytes  at least sdq_fuse_host_workspace_bytes(M, K, chunk_rows)
+ *   chunk_rows       rows per chunk, a multiple of 128 (0 = choose)
+ */
+int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q,
+                  float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M,
+                  int64_t K, int32_t group_size, void* workspace,
+                  size_t workspace_bytes, int64_t chunk_rows, void* stream);
+
+/* Device workspace sdq_fuse_host needs for this shape and chunk size
+ * (chunk_rows = 0: the size it would choose).  0 for invalid arguments. */
+size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows);
+
+/*
+ * sdq_device_status -- synchronizes `stream`, then reads and clears the
+ * device-side status word of the current device: SDQ_OK, or
+ * SDQ_ERR_TIMEOUT if a kernel's wait on its shared-memory pipeline ran past
+ * its limit (the kernel then stops early and its outputs are incomplete).
+ */
+int sdq_device_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* sdq_status_string(int status);
+
+/* cudaError_t of the last CUDA failure seen by this thread (0 if none). */
+int sdq_last_cuda_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* sdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDQ_H_ */

@@ -1,0 +1,113 @@
+"""ctypes binding of libsdq.so (the C ABI in include/sdq.h).
+
+Argument marshalling only: every step of the op runs in the CUDA library.
+There is no CPU path; if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsdq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m swiglu_backward_int8_b200.build` "
+        "(or __graft_entry__.build()); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+
+_lib.sdq_fuse.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P]
+_lib.sdq_fuse.restype = ctypes.c_int
+_lib.sdq_validate.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32]
+_lib.sdq_validate.restype = ctypes.c_int
+_lib.sdq_fuse_host.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P, ctypes.c_size_t, _I64, _P]
+_lib.sdq_fuse_host.restype = ctypes.c_int
+_lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
+_lib.sdq_fuse_host_workspace_bytes.restype = ctypes.c_size_t
+_lib.sdq_device_status.argtypes = [_P]
+_lib.sdq_device_status.restype = ctypes.c_int
+_lib.sdq_status_string.argtypes = [ctypes.c_int]
+_lib.sdq_status_string.restype = ctypes.c_char_p
+_lib.sdq_last_cuda_error.argtypes = []
+_lib.sdq_last_cuda_error.restype = ctypes.c_int
+_lib.sdq_version.argtypes = []
+_lib.sdq_version.restype = ctypes.c_char_p
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    ERR_NULL = 1
+    ERR_GROUP = 2
+    ERR_SHAPE = 3
+    ERR_ALIGN = 4
+    ERR_CUDA = 5
+    ERR_TIMEOUT = 6
+    ERR_WORKSPACE = 7
+
+
+class SdqError(RuntimeError):
+    """A non-OK status from the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = Status(status) if status in Status._value2member_map_ else status
+        msg = f"{where}: {status_string(status)}"
+        if status == Status.ERR_CUDA:
+            msg += f" (cudaError {last_cuda_error()})"
+        super().__init__(msg)
+
+
+def status_string(status: int) -> str:
+    return _lib.sdq_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> int:
+    return int(_lib.sdq_last_cuda_error())
+
+
+def version() -> str:
+    return _lib.sdq_version().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != Status.OK:
+        raise SdqError(status, where)
+
+
+def sdq_fuse(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int, y_s_t: int,
+             M: int, K: int, group_size: int = 128, stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the device entry point (device addresses as ints)."""
+    _check(_lib.sdq_fuse(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                         group_size, stream or 0), "sdq_fuse")
+
+
+def sdq_validate(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                 y_s_t: int, M: int, K: int, group_size: int = 128) -> int:
+    """Argument checks only (no CUDA call); returns the status code."""
+    return int(_lib.sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                 group_size))
+
+
+def sdq_fuse_host(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                  y_s_t: int, M: int, K: int, group_size: int, workspace: int,
+                  workspace_bytes: int, chunk_rows: int = 0, stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the host-buffer entry point."""
+    _check(_lib.sdq_fuse_host(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                              group_size, workspace, workspace_bytes, chunk_rows, stream or 0),
+           "sdq_fuse_host")
+
+
+def sdq_fuse_host_workspace_bytes(M: int, K: int, chunk_rows: int = 0) -> int:
+    return int(_lib.sdq_fuse_host_workspace_bytes(M, K, chunk_rows))
+
+
+def sdq_device_status(stream: Optional[int] = None) -> int:
+    """Synchronize `stream`, read and clear the device status word."""
+    return int(_lib.sdq_device_status(stream or 0))

@@ -1,0 +1,312 @@
+// C ABI of silu_dot_fwd_bwd_quant_fuse (declared in include/sdq.h): argument
+// validation, TMA descriptors, the launch of the fused sm_100a kernel, and the
+// chunked host-buffer path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "sdq.h"
+#include "sdq_kernel.cuh"
+
+namespace {
+
+// Kernel configuration: consumer warps and pipeline depth.
+constexpr int kNW = 8;
+constexpr int kStages = 8;
+using Cfg = sdq::Config<kNW, kStages>;
+
+constexpr int kMaxDevices = 64;
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  cudaGetLastError();  // clear the sticky-free error so the next call starts clean
+  return SDQ_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("SDQ_WAIT_LIMIT_MS");
+    const long long ms = e ? std::atoll(e) : 0;
+    return static_cast<uint64_t>(ms > 0 ? ms : 4000) * 1000000ull;
+  }();
+  return v;
+}
+
+struct DeviceState {
+  std::once_flag init;
+  cudaError_t init_err = cudaSuccess;
+  int sms = 0;
+  // host-buffer pipeline: copy streams and events, guarded by `mu`
+  std::mutex mu;
+  bool pipe_ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in_ready[2] = {}, out_ready[2] = {}, buf_free[2] = {};
+};
+DeviceState g_dev[kMaxDevices];
+
+int current_device(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
+  DeviceState& d = g_dev[dev];
+  std::call_once(d.init, [&d, dev] {
+    d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (d.init_err == cudaSuccess)
+      d.init_err = cudaFuncSetAttribute(sdq::fuse_kernel<kNW, kStages>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(sdq::smem_bytes<kNW, kStages>()));
+  });
+  if (d.init_err != cudaSuccess) return cuda_fail(d.init_err);
+  *out = &d;
+  return SDQ_OK;
+}
+
+int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+             uint64_t row_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(sdq::kG), static_cast<cuuint32_t>(sdq::kSubRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return SDQ_OK;
+}
+
+// Launch on validated arguments (M > 0).
+int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, float* yst,
+           int64_t M, int64_t K, cudaStream_t stream) {
+  DeviceState* d = nullptr;
+  int st = current_device(&d);
+  if (st != SDQ_OK) return st;
+  CUtensorMap mx, mg;
+  if ((st = make_map(&mx, x, 2 * K, M, 4 * K)) != SDQ_OK) return st;
+  if ((st = make_map(&mg, gy, K, M, 2 * K)) != SDQ_OK) return st;
+  sdq::Params p;
+  p.giq = giq;
+  p.gis = gis;
+  p.yqt = yqt;
+  p.yst = yst;
+  p.M = M;
+  p.K = static_cast<int32_t>(K);
+  p.Kg = static_cast<int32_t>(K / sdq::kG);
+  p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
+  p.num_tiles = p.Mg * p.Kg;
+  p.yqt_vec16 = (M % 16 == 0) ? 1 : 0;
+  p.wait_limit_ns = wait_limit_ns();
+  const int grid = std::min(p.num_tiles, d->sms);
+  sdq::fuse_kernel<kNW, kStages><<<grid, Cfg::kThreads, sdq::smem_bytes<kNW, kStages>(), stream>>>(
+      mx, mg, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SDQ_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+struct ChunkLayout {
+  size_t x, gy, giq, gis, yqt, yst, total;  // byte offsets inside one buffer set
+};
+
+ChunkLayout chunk_layout(int64_t CR, int64_t K) {
+  const int64_t Kg = K / sdq::kG;
+  ChunkLayout L;
+  size_t off = 0;
+  L.x = off;   off += align256(size_t(CR) * 2 * K * 2);
+  L.gy = off;  off += align256(size_t(CR) * K * 2);
+  L.giq = off; off += align256(size_t(CR) * 2 * K);
+  L.gis = off; off += align256(size_t(CR) * 2 * Kg * 4);
+  L.yqt = off; off += align256(size_t(K) * CR);
+  L.yst = off; off += align256(size_t(K) * (CR / sdq::kG) * 4);
+  L.total = off;
+  return L;
+}
+
+int64_t choose_chunk_rows(int64_t M, int64_t K) {
+  // Aim for at least four chunks so copies and kernels overlap, with each
+  // chunk's inputs at most ~64 MB.
+  const int64_t by_count = ((M + 3) / 4 + sdq::kG - 1) / sdq::kG * sdq::kG;
+  int64_t by_bytes = (int64_t(64) << 20) / (6 * K) / sdq::kG * sdq::kG;
+  by_bytes = std::max<int64_t>(by_bytes, sdq::kG);
+  return std::max<int64_t>(sdq::kG, std::min(by_count, by_bytes));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sdq_version(void) { return "0.1.0"; }
+
+int sdq_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char* sdq_status_string(int status) {
+  switch (status) {
+    case SDQ_OK: return "SDQ_OK";
+    case SDQ_ERR_NULL: return "SDQ_ERR_NULL: a required pointer is NULL";
+    case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 128";
+    case SDQ_ERR_SHAPE: return "SDQ_ERR_SHAPE: need M >= 0 and K a positive multiple of 128 within the size limits";
+    case SDQ_ERR_ALIGN: return "SDQ_ERR_ALIGN: x, grad_y, grad_input_q, y_q_t need 16-byte and scales 4-byte alignment";
+    case SDQ_ERR_CUDA: return "SDQ_ERR_CUDA: a CUDA call failed (see sdq_last_cuda_error)";
+    case SDQ_ERR_TIMEOUT: return "SDQ_ERR_TIMEOUT: a device-side wait ran past its limit";
+    case SDQ_ERR_WORKSPACE: return "SDQ_ERR_WORKSPACE: workspace too small or misaligned";
+    default: return "SDQ_ERR_UNKNOWN";
+  }
+}
+
+int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
+                 const float* grad_input_s, const int8_t* y_q_t, const float* y_s_t, int64_t M,
+                 int64_t K, int32_t group_size) {
+  if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
+  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
+    return SDQ_ERR_SHAPE;
+  const int64_t tiles = ((M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE) * (K / SDQ_GROUP_SIZE);
+  if (tiles > INT32_MAX) return SDQ_ERR_SHAPE;
+  if (M == 0) return SDQ_OK;
+  if (!x || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t) return SDQ_ERR_NULL;
+  const uintptr_t a16 = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(grad_y) |
+                        reinterpret_cast<uintptr_t>(grad_input_q) | reinterpret_cast<uintptr_t>(y_q_t);
+  const uintptr_t a4 = reinterpret_cast<uintptr_t>(grad_input_s) | reinterpret_cast<uintptr_t>(y_s_t);
+  if ((a16 & 15u) || (a4 & 3u)) return SDQ_ERR_ALIGN;
+  return SDQ_OK;
+}
+
+int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q, float* grad_input_s,
+             int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K, int32_t group_size, void* stream) {
+  const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
+  if (st != SDQ_OK || M == 0) return st;
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                static_cast<cudaStream_t>(stream));
+}
+
+size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows) {
+  if (M < 1 || K < 1 || K % SDQ_GROUP_SIZE != 0 || K > SDQ_MAX_K || M > SDQ_MAX_M) return 0;
+  if (chunk_rows < 0 || chunk_rows % SDQ_GROUP_SIZE != 0) return 0;
+  const int64_t CR = chunk_rows ? chunk_rows : choose_chunk_rows(M, K);
+  return 2 * chunk_layout(CR, K).total;
+}
+
+int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float* grad_input_s,
+                  int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K, int32_t group_size,
+                  void* workspace, size_t workspace_bytes, int64_t chunk_rows, void* stream) {
+  if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
+  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K ||
+      chunk_rows < 0 || chunk_rows % SDQ_GROUP_SIZE != 0)
+    return SDQ_ERR_SHAPE;
+  if (M == 0) return SDQ_OK;
+  if (!x || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t) return SDQ_ERR_NULL;
+  if (!workspace) return SDQ_ERR_NULL;
+  const int64_t CR = chunk_rows ? chunk_rows : choose_chunk_rows(M, K);
+  const ChunkLayout L = chunk_layout(CR, K);
+  if (workspace_bytes < 2 * L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SDQ_ERR_WORKSPACE;
+
+  DeviceState* d = nullptr;
+  int st = current_device(&d);
+  if (st != SDQ_OK) return st;
+  std::lock_guard<std::mutex> lock(d->mu);
+  cudaError_t e = cudaSuccess;
+  if (!d->pipe_ready) {
+    if ((e = cudaStreamCreateWithFlags(&d->h2d, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamCreateWithFlags(&d->d2h, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    cudaEvent_t* evs[] = {&d->start, &d->in_ready[0], &d->in_ready[1], &d->out_ready[0],
+                          &d->out_ready[1], &d->buf_free[0], &d->buf_free[1]};
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+    d->pipe_ready = true;
+  }
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int64_t Kg = K / SDQ_GROUP_SIZE;
+  const int64_t Mg = (M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
+  const auto* xh = static_cast<const uint8_t*>(x);
+  const auto* gh = static_cast<const uint8_t*>(grad_y);
+  auto* ws = static_cast<uint8_t*>(workspace);
+
+#define SDQ_CHECK(call)                         \
+  do {                                          \
+    if ((e = (call)) != cudaSuccess) return cuda_fail(e); \
+  } while (0)
+
+  // Order everything after the work already queued on the caller's stream.
+  SDQ_CHECK(cudaEventRecord(d->start, cs));
+  SDQ_CHECK(cudaStreamWaitEvent(d->h2d, d->start, 0));
+  SDQ_CHECK(cudaStreamWaitEvent(d->d2h, d->start, 0));
+  const int64_t nchunks = (M + CR - 1) / CR;
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int b = static_cast<int>(c & 1);
+    uint8_t* base = ws + b * L.total;
+    const int64_t m0 = c * CR;
+    const int64_t mc = std::min(CR, M - m0);
+    const int64_t mcg = (mc + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
+    // host -> device (after the chunk that last used this buffer set has left)
+    if (c >= 2) SDQ_CHECK(cudaStreamWaitEvent(d->h2d, d->buf_free[b], 0));
+    SDQ_CHECK(cudaMemcpyAsync(base + L.x, xh + m0 * 4 * K, size_t(mc) * 4 * K,
+                              cudaMemcpyHostToDevice, d->h2d));
+    SDQ_CHECK(cudaMemcpyAsync(base + L.gy, gh + m0 * 2 * K, size_t(mc) * 2 * K,
+                              cudaMemcpyHostToDevice, d->h2d));
+    SDQ_CHECK(cudaEventRecord(d->in_ready[b], d->h2d));
+    // kernel on the caller's stream
+    SDQ_CHECK(cudaStreamWaitEvent(cs, d->in_ready[b], 0));
+    st = launch(base + L.x, base + L.gy, reinterpret_cast<int8_t*>(base + L.giq),
+                reinterpret_cast<float*>(base + L.gis), reinterpret_cast<int8_t*>(base + L.yqt),
+                reinterpret_cast<float*>(base + L.yst), mc, K, cs);
+    if (st != SDQ_OK) return st;
+    SDQ_CHECK(cudaEventRecord(d->out_ready[b], cs));
+    // device -> host
+    SDQ_CHECK(cudaStreamWaitEvent(d->d2h, d->out_ready[b], 0));
+    SDQ_CHECK(cudaMemcpyAsync(grad_input_q + m0 * 2 * K, base + L.giq, size_t(mc) * 2 * K,
+                              cudaMemcpyDeviceToHost, d->d2h));
+    SDQ_CHECK(cudaMemcpyAsync(grad_input_s + m0 * 2 * Kg, base + L.gis, size_t(mc) * 2 * Kg * 4,
+                              cudaMemcpyDeviceToHost, d->d2h));
+    SDQ_CHECK(cudaMemcpy2DAsync(y_q_t + m0, size_t(M), base + L.yqt, size_t(mc), size_t(mc),
+                                size_t(K), cudaMemcpyDeviceToHost, d->d2h));
+    SDQ_CHECK(cudaMemcpy2DAsync(y_s_t + m0 / SDQ_GROUP_SIZE, size_t(Mg) * 4, base + L.yst,
+                                size_t(mcg) * 4, size_t(mcg) * 4, size_t(K),
+                                cudaMemcpyDeviceToHost, d->d2h));
+    SDQ_CHECK(cudaEventRecord(d->buf_free[b], d->d2h));
+  }
+  // The caller's stream completes only after the last copies have landed.
+  SDQ_CHECK(cudaStreamWaitEvent(cs, d->buf_free[(nchunks - 1) & 1], 0));
+  if (nchunks > 1) SDQ_CHECK(cudaStreamWaitEvent(cs, d->buf_free[nchunks & 1], 0));
+#undef SDQ_CHECK
+  return SDQ_OK;
+}
+
+int sdq_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, sdq::g_sdq_dev_status, sizeof v)) != cudaSuccess) return cuda_fail(e);
+  if (v) {
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(sdq::g_sdq_dev_status, &zero, sizeof zero)) != cudaSuccess)
+      return cuda_fail(e);
+    return SDQ_ERR_TIMEOUT;
+  }
+  return SDQ_OK;
+}
+
+}  // extern "C"

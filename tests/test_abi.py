@@ -1,0 +1,110 @@
+"""The C ABI library: builds, loads, exports every symbol include/sdq.h
+declares, and its host-side validation answers without a GPU (no compute
+calls here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdq.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sdq_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from swiglu_backward_int8_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("sdq_fuse", "sdq_validate", "sdq_fuse_host", "sdq_fuse_host_workspace_bytes",
+                 "sdq_device_status", "sdq_status_string", "sdq_last_cuda_error", "sdq_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_python_binding_loads():
+    import swiglu_backward_int8_b200 as sdq
+    assert sdq.version() == "0.1.0"
+    assert sdq.status_string(0) == "SDQ_OK"
+    assert "group_size" in sdq.status_string(2)
+
+
+A = 1 << 20  # a 16-byte-aligned fake address: validation never dereferences
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(), 0),
+    (dict(group_size=64), 2),
+    (dict(K=100), 3),
+    (dict(K=0), 3),
+    (dict(M=-1), 3),
+    (dict(K=1 << 21), 3),
+    (dict(x=0), 1),
+    (dict(y_s_t=0), 1),
+    (dict(x=A + 2), 4),
+    (dict(y_q_t=A + 8), 4),
+    (dict(grad_input_s=A + 2), 4),
+    (dict(grad_input_s=A + 4), 0),
+    (dict(M=0, x=0, grad_y=0), 0),
+])
+def test_validation_statuses(args, status):
+    import swiglu_backward_int8_b200 as sdq
+    a = dict(x=A, grad_y=A, grad_input_q=A, grad_input_s=A, y_q_t=A, y_s_t=A, M=256, K=256,
+             group_size=128)
+    a.update(args)
+    assert sdq.sdq_validate(a["x"], a["grad_y"], a["grad_input_q"], a["grad_input_s"], a["y_q_t"],
+                            a["y_s_t"], a["M"], a["K"], a["group_size"]) == status
+
+
+def test_fuse_rejects_before_any_cuda_call():
+    # Invalid arguments return their status without touching CUDA (works on a
+    # machine with no GPU).
+    import swiglu_backward_int8_b200 as sdq
+    with pytest.raises(sdq.SdqError) as ei:
+        sdq.sdq_fuse(A, A, A, A, A, A, 256, 200, 128)
+    assert ei.value.status == sdq.Status.ERR_SHAPE
+    with pytest.raises(sdq.SdqError) as ei:
+        sdq.sdq_fuse(A, A, A, A, A, A, 256, 256, 32)
+    assert ei.value.status == sdq.Status.ERR_GROUP
+    sdq.sdq_fuse(0, 0, 0, 0, 0, 0, 0, 256, 128)  # M == 0: nothing to do
+
+
+def test_host_workspace_sizes():
+    import swiglu_backward_int8_b200 as sdq
+    assert sdq.sdq_fuse_host_workspace_bytes(4096, 1408, 0) > 0
+    assert sdq.sdq_fuse_host_workspace_bytes(4096, 100, 0) == 0
+    assert sdq.sdq_fuse_host_workspace_bytes(4096, 1408, 100) == 0
+    b128 = sdq.sdq_fuse_host_workspace_bytes(4096, 1408, 128)
+    b256 = sdq.sdq_fuse_host_workspace_bytes(4096, 1408, 256)
+    # two buffer sets of chunk_rows * (6K input + 3K output bytes + scales)
+    assert b128 >= 2 * 128 * 1408 * 9 and b256 >= 2 * b128 - 4096
+
+
+def test_torch_wrapper_argument_checks():
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    x = torch.zeros(8, 256, dtype=torch.bfloat16)
+    gy = torch.zeros(8, 128, dtype=torch.bfloat16)
+    outs = sdq.allocate_outputs(8, 128, "cpu")
+    with pytest.raises(ValueError):   # host tensors are not accepted by the device entry
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, *outs)
+    with pytest.raises(ValueError):
+        sdq.silu_dot_fwd_bwd_quant_fuse(x.float(), gy, *outs)
+    with pytest.raises(ValueError):
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy[:, :64], *outs)

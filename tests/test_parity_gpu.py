@@ -1,0 +1,199 @@
+"""CUDA path vs the CPU oracle, element by element, on the same seeded inputs.
+
+Tolerances and their derivation are in tests/gpu_util.py.  Every output is
+surrounded by guard bytes and prefilled with values the op never writes, so
+a case also proves that each element was written exactly where it belongs.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+_STATS = {}
+
+
+def _check(w: W.Workload):
+    x, gy = W.make_inputs(w)
+    got = U.run_cuda(x, gy)
+    ref = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, w.group_size)
+    st = U.compare(got, ref, w.name)
+    _STATS[w.name] = st
+    return got, ref, st
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _report():
+    yield
+    path = os.environ.get("SDQ_PARITY_REPORT")
+    if path:
+        with open(path, "w") as f:
+            json.dump(_STATS, f, indent=1)
+
+
+# The four configurations the oracle finishes in seconds run in full.
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_workload_full(idx):
+    _check(W.WORKLOADS[idx])
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 31, 32, 33, 100, 127, 128, 129, 200, 257, 1000])
+@pytest.mark.parametrize("K", [128, 384])
+def test_odd_and_tail_shapes(M, K):
+    _check(W.small_workload(M, K, seed=M * 7 + K))
+
+
+def test_saturated_and_tiny_values():
+    # |gate| up to ~150 (sigma saturates to 0 / 1), tiny grad_y
+    _check(W.small_workload(300, 256, seed=17, sigma_x=30.0, sigma_grad_y=1e-6))
+    _check(W.small_workload(300, 256, seed=18, sigma_x=1.0, sigma_grad_y=3.0,
+                            outlier_frac=0.02, outlier_mult=50.0))
+
+
+def test_zero_groups_on_both_axes():
+    M, K = 300, 384
+    x, gy = W.make_inputs(W.small_workload(M, K, seed=21))
+    x[:128, 128:256] = 0           # gate = 0 -> y = 0 for tokens 0..127, channels 128..255
+    x[200, :] = 0                  # token 200: gate = up = 0 -> both row halves all-zero
+    x[:, K + 300] = 0              # up = 0 in one channel: y = 0 and d_gate = 0 there
+    got = U.run_cuda(x, gy)
+    ref = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy)
+    U.compare(got, ref, "zero groups")
+    giq, gis, yqt, yst = got
+    assert np.all(yst[128:256, 0] == 1.0) and not yqt[128:256, :128].any()
+    assert np.all(gis[200] == 1.0) and not giq[200].any()
+
+
+def test_outlier_workload_zero_row_groups():
+    w = W.WORKLOADS[3]
+    x, gy = W.make_inputs(w)
+    giq, gis, yqt, yst = U.run_cuda(x, gy)
+    for r, j in W.zero_group_positions(w):
+        assert gis[r, j] == 1.0 and gis[r, w.Kg + j] == 1.0
+        assert not giq[r, j * 128:(j + 1) * 128].any()
+        assert not giq[r, w.K + j * 128:w.K + (j + 1) * 128].any()
+
+
+def test_deterministic_and_on_a_side_stream():
+    w = W.small_workload(515, 256, seed=5)
+    x, gy = W.make_inputs(w)
+    a = U.run_cuda(x, gy)
+    s = torch.cuda.Stream()
+    b = U.run_cuda(x, gy, stream=s)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_m_zero_is_a_noop():
+    import swiglu_backward_int8_b200 as sdq
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    gy = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    outs = sdq.allocate_outputs(0, 128, "cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, *outs)
+    torch.cuda.synchronize()
+
+
+def test_misaligned_input_is_rejected_and_nothing_written():
+    import swiglu_backward_int8_b200 as sdq
+    M, K = 128, 128
+    base = torch.zeros(M * 2 * K + 8, dtype=torch.bfloat16, device="cuda")
+    x = base[1:1 + M * 2 * K].view(M, 2 * K)          # 2-byte offset
+    gy = torch.zeros(M, K, dtype=torch.bfloat16, device="cuda")
+    outs = [torch.full(s, -128 if i % 2 == 0 else -1, dtype=dt, device="cuda")
+            for i, (s, dt) in enumerate(zip(sdq.output_shapes(M, K),
+                                            (torch.int8, torch.float32, torch.int8, torch.float32)))]
+    with pytest.raises(sdq.SdqError) as ei:
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, *outs)
+    assert ei.value.status == sdq.Status.ERR_ALIGN
+    torch.cuda.synchronize()
+    assert (outs[0] == -128).all() and (outs[1] == -1).all()
+
+
+@pytest.mark.parametrize("M,K,chunk", [(4096, 1408, 0), (4000, 2048, 1024), (1000, 256, 256),
+                                       (77, 128, 0)])
+def test_host_buffer_entry_matches_device_entry(M, K, chunk):
+    import swiglu_backward_int8_b200 as sdq
+    x, gy = W.make_inputs(W.small_workload(M, K, seed=M + K))
+    dev = U.run_cuda(x, gy)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    gyh = torch.from_numpy(gy.view(np.int16)).view(torch.bfloat16).pin_memory()
+    outs = [t.pin_memory() for t in sdq.allocate_outputs(M, K, "cpu")]
+    for t in outs:
+        t.fill_(-128 if t.dtype == torch.int8 else float("nan"))
+    ws = torch.empty(sdq.sdq_fuse_host_workspace_bytes(M, K, chunk), dtype=torch.uint8, device="cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse_host(xh, gyh, *outs, workspace=ws, chunk_rows=chunk)
+    for a, b in zip(dev, outs):
+        assert np.array_equal(a, b.numpy())
+    # pageable host memory works too
+    outs2 = sdq.allocate_outputs(M, K, "cpu")
+    sdq.silu_dot_fwd_bwd_quant_fuse_host(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16),
+                                         torch.from_numpy(gy.view(np.int16)).view(torch.bfloat16),
+                                         *outs2, workspace=ws, chunk_rows=chunk)
+    for a, b in zip(dev, outs2):
+        assert np.array_equal(a, b.numpy())
+
+
+def test_host_entry_rejects_small_workspace():
+    import swiglu_backward_int8_b200 as sdq
+    M, K = 256, 256
+    x = torch.zeros(M, 2 * K, dtype=torch.bfloat16)
+    gy = torch.zeros(M, K, dtype=torch.bfloat16)
+    outs = sdq.allocate_outputs(M, K, "cpu")
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sdq.SdqError) as ei:
+        sdq.silu_dot_fwd_bwd_quant_fuse_host(x, gy, *outs, workspace=ws)
+    assert ei.value.status == sdq.Status.ERR_WORKSPACE
+
+
+def _tiles_to_sample(Mg, Kg, n, seed):
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0), (Mg - 1, Kg - 1), (0, Kg - 1), (Mg - 1, 0)}
+    while len(picks) < n:
+        picks.add((int(rng.integers(Mg)), int(rng.integers(Kg))))
+    return sorted(picks)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("idx", [4, 2])
+def test_full_size_sampled_tiles_and_invariants(idx):
+    """Full-size workloads in the bench's launch configuration: sampled tiles
+    against the oracle (each tile holds whole groups on both axes), and
+    properties that hold at any size checked over every element."""
+    import swiglu_backward_int8_b200 as sdq
+    w = W.WORKLOADS[idx]
+    x, gy = W.make_inputs(w)
+    M, K, G = w.M, w.K, 128
+    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
+    outs = sdq.allocate_outputs(M, K, "cuda")
+    for t in outs:
+        t.fill_(U.SENTINEL_Q if t.dtype == torch.int8 else float("nan"))
+    sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *outs)
+    torch.cuda.synchronize()
+    assert sdq.sdq_device_status() == 0
+    giq, gis, yqt, yst = outs
+    # every element written; scales finite and positive
+    assert not (giq == U.SENTINEL_Q).any() and not (yqt == U.SENTINEL_Q).any()
+    assert torch.isfinite(gis).all() and (gis > 0).all()
+    assert torch.isfinite(yst).all() and (yst > 0).all()
+    # each group's largest |q| is 127 unless the group is all zero (scale 1, q 0)
+    rmax = giq.view(M, 2 * w.Kg, G).abs().amax(dim=2)
+    assert ((rmax == 127) | ((rmax == 0) & (gis == 1))).all()
+    cmax = yqt.view(K, M // G, G).abs().amax(dim=2)
+    assert ((cmax == 127) | ((cmax == 0) & (yst == 1))).all()
+    host = [t.cpu().numpy() for t in outs]
+    n_diff = 0
+    for (i, j) in _tiles_to_sample(w.Mg, w.Kg, 40, seed=idx):
+        ref = U.oracle_tile(x, gy, i, j)
+        got = U.tile_of(host, M, K, i, j)
+        st = U.compare(got, ref, f"{w.name} tile ({i},{j})")
+        n_diff += st["grad_input_q"]["n_diff"] + st["y_q_t"]["n_diff"]
+    _STATS[w.name + " (40 sampled tiles)"] = {"int8_n_diff": n_diff}

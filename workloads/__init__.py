@@ -24,8 +24,10 @@ quantization op described on "kernelgen-challenge-9-task3-silu-quant"
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from typing import Dict, List, Tuple
 
 import numpy as np
@@ -104,14 +106,28 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def _threads() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
+
+
 def normal_bf16(seed: int, stream: int, count: int, sigma: float) -> np.ndarray:
-    """``count`` samples of N(0, sigma) as bf16 bits, generated in chunks."""
+    """``count`` samples of N(0, sigma) as bf16 bits, generated in chunks
+    (on several threads; the values do not depend on the chunking)."""
     key = stream_key(seed, stream)
     out = np.empty(count, dtype=np.uint16)
-    for s in range(0, count, _CHUNK):
+
+    def fill(s: int) -> None:
         n = min(_CHUNK, count - s)
         z = normals(key, s, n) * float(sigma)
         out[s:s + n] = f32_to_bf16_bits(z.astype(np.float32))
+
+    starts = range(0, count, _CHUNK)
+    if count > _CHUNK and _threads() > 1:
+        with concurrent.futures.ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(fill, starts))
+    else:
+        for s in starts:
+            fill(s)
     return out
 
 
