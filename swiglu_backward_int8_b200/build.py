@@ -1,6 +1,8 @@
 """Build the in-tree CUDA library ``libsdq.so`` for sm_100a.
 
-    python -m swiglu_backward_int8_b200.build [--verbose]
+    python swiglu_backward_int8_b200/build.py [--verbose]
+
+(run it as a script: importing the package needs the library it builds)
 
 nvcc compiles ``csrc/sdq_api.cu`` (host API + the fused kernel) into a shared
 library with a C ABI (``include/sdq.h``); the CUDA runtime is linked

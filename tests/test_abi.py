@@ -21,8 +21,8 @@ def _declared_functions():
 
 @pytest.fixture(scope="module")
 def lib():
-    from swiglu_backward_int8_b200 import build
-    path = build.build()
+    import __graft_entry__
+    path = __graft_entry__._build_module().build()
     return ctypes.CDLL(path)
 
 
