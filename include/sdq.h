@@ -62,7 +62,8 @@ typedef enum sdq_status {
                             scale pointer not 4-byte aligned                          */
   SDQ_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed (see sdq_last_cuda_error) */
   SDQ_ERR_TIMEOUT = 6,   /* a device-side wait hit its time limit (sdq_device_status) */
-  SDQ_ERR_WORKSPACE = 7  /* the workspace given to sdq_fuse_host is too small        */
+  SDQ_ERR_WORKSPACE = 7, /* the workspace given to sdq_fuse_host is too small        */
+  SDQ_ERR_TOO_LARGE = 8  /* sdq_fuse_host_noalloc: K too large for its fixed scratch  */
 } sdq_status;
 
 /* Largest accepted sizes: M < 2^31 (tensor-map coordinates are 32-bit) and
@@ -119,6 +120,44 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q,
 /* Device workspace sdq_fuse_host needs for this shape and chunk size
  * (chunk_rows = 0: the size it would choose).  0 for invalid arguments. */
 size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows);
+
+/*
+ * sdq_fuse_host_noalloc -- sdq_fuse_host for callers that cannot allocate
+ * device memory.  (The page has no counterpart: this entry exists for
+ * callers of this library, not for the method.)
+ *
+ * Who needs it: code that holds no device allocator of its own or must not
+ * call one -- a plain C/C++ host program that only has host buffers, a
+ * plugin inside a framework whose caching allocator owns all device memory
+ * (a cudaMalloc behind its back can fail or fragment the pool), or a service
+ * that forbids device allocation after start-up.  Such a caller cannot
+ * provide the workspace that sdq_fuse_host asks for.
+ *
+ * Same arguments, shapes, layouts and results as sdq_fuse_host, minus the
+ * workspace.  The staging buffers live in one fixed device array of
+ * SDQ_NOALLOC_SCRATCH_BYTES inside this library (every GPU that loads the
+ * library holds it until the process exits).  The rows go through it in
+ * chunks of a multiple of 128 rows, as many as fit; host->device copy,
+ * kernel and device->host copy of each chunk are queued on `stream` alone.
+ * The call allocates nothing: no cudaMalloc/cudaFree, no stream or event
+ * creation.
+ *   - Limit: a 128-row chunk must fit, i.e. K <= SDQ_NOALLOC_MAX_K; larger K
+ *     returns SDQ_ERR_TOO_LARGE before any CUDA call.  M is unlimited.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Sharing: all calls on a device share the one array, and it keeps the
+ *     last call's contents (every byte a call reads is written by that same
+ *     call first, so nothing needs clearing).  Calls that overlap on the GPU
+ *     (on different streams, or from different threads) race on the array:
+ *     serialize them.
+ *   - Host outputs are complete once `stream` has been synchronized.
+ */
+#define SDQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define SDQ_NOALLOC_MAX_K 28800LL
+int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_q,
+                          float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M,
+                          int64_t K, int32_t group_size, void* stream);
 
 /*
  * sdq_device_status -- synchronizes `stream`, then reads and clears the

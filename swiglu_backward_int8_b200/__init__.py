@@ -17,12 +17,13 @@ from typing import Optional, Tuple
 import torch
 
 from ._lib import (LIB_PATH, SdqError, Status, last_cuda_error, sdq_device_status, sdq_fuse,
-                   sdq_fuse_host, sdq_fuse_host_workspace_bytes, sdq_validate, status_string,
-                   version)
+                   sdq_fuse_host, sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes,
+                   sdq_validate, status_string, version)
 
 __all__ = [
     "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs",
-    "output_shapes", "sdq_fuse", "sdq_fuse_host", "sdq_fuse_host_workspace_bytes", "sdq_validate",
+    "output_shapes", "sdq_fuse", "sdq_fuse_host", "sdq_fuse_host_noalloc",
+    "sdq_fuse_host_workspace_bytes", "sdq_validate",
     "sdq_device_status", "SdqError", "Status", "status_string", "last_cuda_error", "version",
     "LIB_PATH", "GROUP_SIZE",
 ]

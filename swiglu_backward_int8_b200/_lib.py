@@ -32,6 +32,8 @@ _lib.sdq_fuse_host.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P, cty
 _lib.sdq_fuse_host.restype = ctypes.c_int
 _lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
 _lib.sdq_fuse_host_workspace_bytes.restype = ctypes.c_size_t
+_lib.sdq_fuse_host_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P]
+_lib.sdq_fuse_host_noalloc.restype = ctypes.c_int
 _lib.sdq_device_status.argtypes = [_P]
 _lib.sdq_device_status.restype = ctypes.c_int
 _lib.sdq_status_string.argtypes = [ctypes.c_int]
@@ -51,6 +53,7 @@ class Status(enum.IntEnum):
     ERR_CUDA = 5
     ERR_TIMEOUT = 6
     ERR_WORKSPACE = 7
+    ERR_TOO_LARGE = 8
 
 
 class SdqError(RuntimeError):
@@ -102,6 +105,17 @@ def sdq_fuse_host(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q
     _check(_lib.sdq_fuse_host(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                               group_size, workspace, workspace_bytes, chunk_rows, stream or 0),
            "sdq_fuse_host")
+
+
+def sdq_fuse_host_noalloc(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                          y_s_t: int, M: int, K: int, group_size: int = 128,
+                          stream: Optional[int] = None) -> None:
+    """Host-buffer entry point for callers that cannot allocate device
+    memory: it stages through a fixed array inside the library instead of a
+    caller workspace (K up to SDQ_NOALLOC_MAX_K = 28800).  Host addresses as
+    ints; the outputs are complete once `stream` is synchronized."""
+    _check(_lib.sdq_fuse_host_noalloc(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                      group_size, stream or 0), "sdq_fuse_host_noalloc")
 
 
 def sdq_fuse_host_workspace_bytes(M: int, K: int, chunk_rows: int = 0) -> int:

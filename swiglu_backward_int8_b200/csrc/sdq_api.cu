@@ -173,6 +173,7 @@ const char* sdq_status_string(int status) {
     case SDQ_ERR_CUDA: return "SDQ_ERR_CUDA: a CUDA call failed (see sdq_last_cuda_error)";
     case SDQ_ERR_TIMEOUT: return "SDQ_ERR_TIMEOUT: a device-side wait ran past its limit";
     case SDQ_ERR_WORKSPACE: return "SDQ_ERR_WORKSPACE: workspace too small or misaligned";
+    case SDQ_ERR_TOO_LARGE: return "SDQ_ERR_TOO_LARGE: K exceeds what fits in the fixed scratch of sdq_fuse_host_noalloc (SDQ_NOALLOC_MAX_K)";
     default: return "SDQ_ERR_UNKNOWN";
   }
 }
@@ -292,6 +293,96 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
   SDQ_CHECK(cudaStreamWaitEvent(cs, d->buf_free[(nchunks - 1) & 1], 0));
   if (nchunks > 1) SDQ_CHECK(cudaStreamWaitEvent(cs, d->buf_free[nchunks & 1], 0));
 #undef SDQ_CHECK
+  return SDQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Staging area of sdq_fuse_host_noalloc: one chunk of x and grad_y and of the
+// four outputs.  In host code this name is only a stand-in; the kernel gets
+// the device address looked up per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SDQ_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocDevice {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  uint8_t* ptr = nullptr;
+};
+NoallocDevice g_noalloc[kMaxDevices];
+
+// Largest multiple of 128 rows whose single buffer set fits in the array.
+int64_t noalloc_chunk_rows(int64_t K) {
+  int64_t rows = 0;
+  for (int64_t cr = SDQ_GROUP_SIZE; chunk_layout(cr, K).total <= SDQ_NOALLOC_SCRATCH_BYTES;
+       cr += SDQ_GROUP_SIZE)
+    rows = cr;
+  return rows;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_q,
+                          float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K,
+                          int32_t group_size, void* stream) {
+  if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
+  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
+    return SDQ_ERR_SHAPE;
+  if (K > SDQ_NOALLOC_MAX_K) return SDQ_ERR_TOO_LARGE;
+  if (M == 0) return SDQ_OK;
+  if (!x || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t) return SDQ_ERR_NULL;
+  const int64_t max_rows = noalloc_chunk_rows(K);
+  if (max_rows < SDQ_GROUP_SIZE) return SDQ_ERR_TOO_LARGE;
+  const int64_t CR = std::min(max_rows, (M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE * SDQ_GROUP_SIZE);
+  const ChunkLayout L = chunk_layout(CR, K);
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
+  NoallocDevice& nd = g_noalloc[dev];
+  std::call_once(nd.once, [&nd] {
+    nd.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&nd.ptr), g_noalloc_scratch);
+  });
+  if (nd.err != cudaSuccess) return cuda_fail(nd.err);
+  uint8_t* base = nd.ptr;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int64_t Kg = K / SDQ_GROUP_SIZE;
+  const int64_t Mg = (M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
+  const auto* xh = static_cast<const uint8_t*>(x);
+  const auto* gh = static_cast<const uint8_t*>(grad_y);
+  for (int64_t m0 = 0; m0 < M; m0 += CR) {
+    const int64_t mc = std::min(CR, M - m0);
+    const int64_t mcg = (mc + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
+    if ((e = cudaMemcpyAsync(base + L.x, xh + m0 * 4 * K, size_t(mc) * 4 * K,
+                             cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(base + L.gy, gh + m0 * 2 * K, size_t(mc) * 2 * K,
+                             cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+      return cuda_fail(e);
+    const int st = launch(base + L.x, base + L.gy, reinterpret_cast<int8_t*>(base + L.giq),
+                          reinterpret_cast<float*>(base + L.gis),
+                          reinterpret_cast<int8_t*>(base + L.yqt),
+                          reinterpret_cast<float*>(base + L.yst), mc, K, cs);
+    if (st != SDQ_OK) return st;
+    if ((e = cudaMemcpyAsync(grad_input_q + m0 * 2 * K, base + L.giq, size_t(mc) * 2 * K,
+                             cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(grad_input_s + m0 * 2 * Kg, base + L.gis, size_t(mc) * 2 * Kg * 4,
+                             cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpy2DAsync(y_q_t + m0, size_t(M), base + L.yqt, size_t(mc), size_t(mc),
+                               size_t(K), cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpy2DAsync(y_s_t + m0 / SDQ_GROUP_SIZE, size_t(Mg) * 4, base + L.yst,
+                               size_t(mcg) * 4, size_t(mcg) * 4, size_t(K),
+                               cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+      return cuda_fail(e);
+  }
   return SDQ_OK;
 }
 
