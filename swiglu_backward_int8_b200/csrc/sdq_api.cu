@@ -15,10 +15,12 @@
 
 namespace {
 
-// Kernel configuration: consumer warps and pipeline depth.
-constexpr int kNW = 8;
-constexpr int kStages = 8;
-using Cfg = sdq::Config<kNW, kStages>;
+// Pipeline depth of the kernel's shared-memory ring (48 KB per stage;
+// compile-time overridable for tuning sweeps).
+#ifndef SDQ_STAGES
+#define SDQ_STAGES 3
+#endif
+constexpr int kStages = SDQ_STAGES;
 
 constexpr int kMaxDevices = 64;
 thread_local int t_last_cuda_error = 0;
@@ -73,9 +75,14 @@ int current_device(DeviceState** out) {
   std::call_once(d.init, [&d, dev] {
     d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     if (d.init_err == cudaSuccess)
-      d.init_err = cudaFuncSetAttribute(sdq::fuse_kernel<kNW, kStages>,
+      d.init_err = cudaFuncSetAttribute(sdq::fuse_kernel<kStages>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(sdq::smem_bytes<kNW, kStages>()));
+                                        static_cast<int>(sdq::smem_bytes<kStages>()));
+    int blocks = 0;
+    if (d.init_err == cudaSuccess)
+      d.init_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &blocks, sdq::fuse_kernel<kStages>, sdq::kThreads, sdq::smem_bytes<kStages>());
+    if (d.init_err == cudaSuccess && blocks < 1) d.init_err = cudaErrorLaunchOutOfResources;
   });
   if (d.init_err != cudaSuccess) return cuda_fail(d.init_err);
   *out = &d;
@@ -88,7 +95,7 @@ int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(sdq::kG), static_cast<cuuint32_t>(sdq::kSubRows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(sdq::kG), static_cast<cuuint32_t>(sdq::kStageRows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -119,8 +126,7 @@ int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, 
   p.yqt_vec16 = (M % 16 == 0) ? 1 : 0;
   p.wait_limit_ns = wait_limit_ns();
   const int grid = std::min(p.num_tiles, d->sms);
-  sdq::fuse_kernel<kNW, kStages><<<grid, Cfg::kThreads, sdq::smem_bytes<kNW, kStages>(), stream>>>(
-      mx, mg, p);
+  sdq::fuse_kernel<kStages><<<grid, sdq::kThreads, sdq::smem_bytes<kStages>(), stream>>>(mx, mg, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return SDQ_OK;

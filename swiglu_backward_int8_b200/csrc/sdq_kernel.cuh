@@ -9,36 +9,40 @@
 //
 // Work decomposition.  A 128-token x 128-channel tile (i, j) holds exactly one
 // quantization group on both axes, so tiles are independent.  The grid is
-// persistent (at most one CTA per SM); CTA b walks tiles b, b + grid, ...
-// in a banded order (8 tile rows per band, tile row fastest) so that the
-// scale sectors of neighbouring tiles are written close together in time.
+// persistent (at most one CTA per SM); CTA b walks tiles b, b + grid, ... in a
+// banded order (8 tile rows per band, tile row fastest) so that the scale
+// sectors of neighbouring tiles are written close together in time.
 //
-// Inside a CTA:
-//   * one producer thread streams each tile as four 32-row sub-tiles; a
-//     sub-tile is three TMA boxes (gate, up, grad_y; 32 x 128 bf16 each,
-//     24 KB) into a STAGES-deep shared-memory ring guarded by full/empty
-//     mbarriers.  Rows past M are zero-filled by the TMA unit, and zeros never
-//     change an amax, so the tail token group is quantized over exactly the
-//     tokens it holds.
-//   * NW consumer warps read a stage into registers and release it at once.
-//     A half-warp owns one token row of the stage, 8 channels per lane:
-//     fp32 math, bf16 rounding, the row amax of d_gate and d_up by a 4-step
-//     shuffle reduction on packed bf16 pairs, scales (amax/127, correctly
-//     rounded) computed once per (row, half) by one lane each, quantization
-//     by multiplication with the inverse scale, 8-byte coalesced stores.
-//   * the bf16 y values stay in registers for the whole tile; the column amax
-//     is reduced in registers, across the two half-warps by one shuffle and
-//     across warps through shared memory.  After the 128 column scales, each
-//     lane quantizes its y values and writes them transposed into an int8
-//     staging tile (row = channel) whose 4-byte words are XOR-swizzled by
-//     channel so the byte-column writes are bank-conflict free; the tile then
-//     leaves as 16-byte stores, each 8-lane group writing one 128-byte line
-//     of y_q_t.
+// Inside a CTA (16 warps, all of them compute):
+//   * each tile arrives as two 64-row stages; a stage is three TMA boxes
+//     (gate, up, grad_y; 64 x 128 bf16 each, 48 KB) in a STAGES-deep
+//     shared-memory ring.  Load n of a CTA is tile n/2, half n%2, so any thread
+//     can issue any load.  Each slot has an mbarrier (TMA byte count); the
+//     warps release a slot through a shared counter and the warp that releases
+//     it last issues the load that goes next into it -- there is no producer
+//     warp, so every warp computes and may use 128 registers.
+//     Rows past M are zero-filled by the TMA unit, and zeros never change an
+//     amax, so a tail token group is quantized over exactly the tokens it holds.
+//   * row pass: a lane owns 16 channels of one token row per stage (8 lanes per
+//     row, 4 rows per warp): fp32 math in packed f32x2 instructions, bf16
+//     rounding, the row amax of d_gate and d_up by a 3-step shuffle reduction
+//     on packed bf16 pairs, the warp's 8 row scales computed by lanes 0-7 at
+//     once and shuffled back, quantization by multiplication with the inverse
+//     scale, coalesced stores; the bf16 y values go to a shared [token][channel]
+//     tile (double-buffered across tiles).
+//   * column pass, after one barrier per tile: a thread owns 2 channels x 16
+//     tokens of that tile, reduces the column amax over the 8 threads that
+//     share its channels, computes the two column scales, quantizes its 32 y
+//     values and stores two 16-byte pieces of y_q_t rows; each group of 8
+//     threads writes one 128-byte line.
+//   * shared-memory layouts are chosen for conflict-free access: a lane of the
+//     upper half of an 8-lane row group takes its two 16-byte chunks in the
+//     opposite order, and the y tile's chunks are XOR-swizzled by token.
 //
 // Every wait on an mbarrier is bounded (Params::wait_limit_ns).  A wait that
-// runs out sets the device status word; the consumers agree on stopping at the
-// next tile boundary through a barrier-reduction, and the producer waits
-// (bounded) for its own in-flight copies before it returns.
+// runs out sets the device status word; the warps agree on stopping at the
+// next tile boundary through a barrier-reduction, and one thread waits
+// (bounded) for the copies still in flight before the CTA exits.
 #pragma once
 
 #include <cstdint>
@@ -47,11 +51,15 @@
 
 namespace sdq {
 
-constexpr int kG = 128;                               // group size = tile edge
-constexpr int kSubRows = 32;                          // token rows per pipeline stage
-constexpr int kNumSub = kG / kSubRows;                // stages per tile
-constexpr int kTensorStageBytes = kSubRows * kG * 2;  // one bf16 box: 8 KB
-constexpr int kStageBytes = 3 * kTensorStageBytes;    // gate + up + grad_y
+constexpr int kG = 128;                             // group size = tile edge
+constexpr int kStageRows = 64;                      // token rows per pipeline stage
+constexpr int kStagesPerTile = kG / kStageRows;     // 2
+constexpr int kBoxBytes = kStageRows * kG * 2;      // one bf16 box: 16 KB
+constexpr int kStageBytes = 3 * kBoxBytes;          // gate + up + grad_y
+constexpr int kYBytes = kG * kG * 2;                // bf16 y tile: 32 KB
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowsPerWarp = kStageRows / kWarps;   // 4 (8 lanes per row)
 
 constexpr int kDevTimeout = 1;  // bit in the device status word
 
@@ -72,28 +80,19 @@ struct Params {
   uint64_t wait_limit_ns;
 };
 
-template <int NW, int STAGES>
-struct Config {
-  static constexpr int kConsumerWarps = NW;
-  static constexpr int kConsumers = NW * 32;
-  static constexpr int kThreads = kConsumers + 32;       // + one producer warp
-  static constexpr int kRowsPerLane = kSubRows / (2 * NW);
-  static_assert(kRowsPerLane >= 1 && kRowsPerLane * 2 * NW == kSubRows, "NW must divide 16");
-};
-
-template <int NW, int STAGES>
+template <int STAGES>
 struct Smem {
-  alignas(128) uint8_t ring[STAGES][kStageBytes];  // [gate | up | grad_y], each [32][128] bf16
-  alignas(16) uint8_t yt[kG * kG];                 // int8 y^T: row = channel, 4-byte words swizzled
-  alignas(16) uint16_t colmax[NW][kG];             // per-warp column amax (bf16 bits)
-  alignas(16) float inv_y[kG];                     // 1 / column scale
+  alignas(128) uint8_t ring[STAGES][kStageBytes];  // [gate | up | grad_y], each [64][128] bf16
+  alignas(16) uint8_t ytile[2][kYBytes];           // bf16 y [token][channel], chunks swizzled
+  alignas(16) float2 scale_tab[128];               // (fl((1+m/128)/127), 1/that) per bf16 mantissa m
   alignas(8) uint64_t full[STAGES];
-  alignas(8) uint64_t empty[STAGES];
+  int released[STAGES];                            // warps done with the slot's current load
+  int issued;                                      // loads issued so far (for the drain on abort)
 };
 
-template <int NW, int STAGES>
+template <int STAGES>
 constexpr size_t smem_bytes() {
-  return sizeof(Smem<NW, STAGES>) + 128;  // + room to align the base to 128 B
+  return sizeof(Smem<STAGES>) + 128;  // + room to align the base to 128 B
 }
 
 // Tile t -> (token-group i, channel-group j), banded: 8 tile rows per band,
@@ -107,297 +106,338 @@ __device__ __forceinline__ void tile_ij(int t, int Mg, int Kg, int& i, int& j) {
   j = r / rows;
 }
 
-// One element: y = silu(g)*u, d_gate = dy*u*silu'(g), d_up = dy*silu(g), fp32.
-__device__ __forceinline__ void swiglu_bwd(float g, float u, float dy, float& y, float& dg,
-                                           float& du) {
-  const float sg = __fdividef(1.0f, 1.0f + __expf(-g));  // sigma(g); 0 or 1 when saturated
-  const float silu = g * sg;
-  y = silu * u;
-  dg = (dy * u) * (sg * fmaf(g, 1.0f - sg, 1.0f));
-  du = dy * silu;
+// Load n of this CTA: stage n % 2 of its (n / 2)-th tile, into slot n % STAGES.
+template <int STAGES>
+__device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* mx,
+                                           const CUtensorMap* mg, const Params& p, uint32_t n,
+                                           uint64_t pol) {
+  const int t = blockIdx.x + static_cast<int>(n / kStagesPerTile) * gridDim.x;
+  int i, j;
+  tile_ij(t, p.Mg, p.Kg, i, j);
+  const int r = i * kG + static_cast<int>(n % kStagesPerTile) * kStageRows;
+  const uint32_t slot = n % STAGES;
+  const uint32_t fb = smem_u32(&s.full[slot]);
+  mbar_arrive_expect_tx(fb, kStageBytes);
+  const uint32_t dst = smem_u32(s.ring[slot]);
+  tma_load_2d(dst, mx, fb, j * kG, r, pol);                          // gate
+  tma_load_2d(dst + kBoxBytes, mx, fb, p.K + j * kG, r, pol);        // up
+  tma_load_2d(dst + 2 * kBoxBytes, mg, fb, j * kG, r, pol);          // grad_y
 }
 
-// Scale and inverse scale of a group from its amax: amax/127 correctly
-// rounded; an all-zero group gets scale 1.
-__device__ __forceinline__ void group_scale(float amax, float& scale, float& inv) {
-  scale = 1.0f;
-  inv = 1.0f;
-  if (amax != 0.0f) {
-    scale = __fdiv_rn(amax, 127.0f);
-    inv = __frcp_rn(scale);
+// bf16 pair -> two floats (exact).
+__device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_lo(v), bf16_hi(v)); }
+
+// Two elements: y = silu(g)*u, d_gate = dy*u*silu'(g), d_up = dy*silu(g) in
+// fp32 (packed pairs), with silu'(g) = sigma(g)*(1 + g*(1 - sigma(g)))
+// = silu*(1 - sigma) + sigma.  Results as bf16 pairs.
+__device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t dw, uint32_t& y,
+                                            uint32_t& dg, uint32_t& du) {
+  const float2 g = unpack2(gw), u = unpack2(uw), dy = unpack2(dw);
+  const float2 one = make_float2(1.0f, 1.0f);
+  const float2 d = __fadd2_rn(make_float2(__expf(-g.x), __expf(-g.y)), one);
+  const float2 sg = make_float2(__fdividef(1.0f, d.x), __fdividef(1.0f, d.y));  // 0 or 1 when saturated
+  const float2 silu = __fmul2_rn(g, sg);
+  const float2 oms = __ffma2_rn(sg, make_float2(-1.0f, -1.0f), one);
+  const float2 dsilu = __ffma2_rn(silu, oms, sg);
+  const float2 yy = __fmul2_rn(silu, u);
+  const float2 gg = __fmul2_rn(__fmul2_rn(dy, u), dsilu);
+  const float2 uu = __fmul2_rn(dy, silu);
+  y = pack_bf16x2(yy.x, yy.y);
+  dg = pack_bf16x2(gg.x, gg.y);
+  du = pack_bf16x2(uu.x, uu.y);
+}
+
+// Scale and inverse scale of a group from its amax, given as non-negative
+// bf16 bits: scale = amax/127 correctly rounded, inv = 1/scale correctly
+// rounded; an all-zero group gets scale 1.  A bf16 amax is (1 + m/128) * 2^e,
+// so scale = fl((1 + m/128)/127) * 2^e exactly whenever that is a normal
+// float: the table holds the two mantissa-dependent quotients and the power of
+// two goes into the exponent field.
+// Tiny groups (amax < 2^-119, bf16 exponent field < 8) take the quotients
+// directly; their 1/scale can exceed the float range, so for them the
+// returned inverse is meant for values pre-multiplied by kTinyPre (= 2^64) and
+// comes back negated as a marker: (v * 2^64) * fl(1/(scale * 2^64)) is the
+// same real number as v * fl(1/scale).
+constexpr float kTinyPre = 18446744073709551616.0f;  // 2^64
+
+__device__ __forceinline__ void group_scale(uint32_t abits, const float2* tab, float& scale,
+                                            float& inv_marked) {
+  const uint32_t ex = abits >> 7;
+  if (ex >= 8u) {
+    const float2 t = tab[abits & 127u];
+    const int sh = (static_cast<int>(ex) - 127) << 23;
+    scale = __int_as_float(__float_as_int(t.x) + sh);
+    inv_marked = __int_as_float(__float_as_int(t.y) - sh);
+  } else if (abits != 0u) {
+    scale = __fdiv_rn(__uint_as_float(abits << 16), 127.0f);
+    inv_marked = -__frcp_rn(scale * kTinyPre);
+  } else {
+    scale = 1.0f;
+    inv_marked = 1.0f;
   }
 }
 
-template <int NW, int STAGES>
-__device__ __forceinline__ void producer(Smem<NW, STAGES>& s, const CUtensorMap* mx,
-                                         const CUtensorMap* mg, const Params& p) {
-  prefetch_tensormap(mx);
-  prefetch_tensormap(mg);
-  const uint64_t pol = l2_policy_evict_first();  // inputs are read exactly once
-  uint32_t n = 0;                                // stages issued
-  bool ok = true;
-  for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-    int i, j;
-    tile_ij(t, p.Mg, p.Kg, i, j);
-    const int64_t row0 = int64_t(i) * kG;
-    const int valid = static_cast<int>((p.M - row0 < kG ? p.M - row0 : int64_t(kG)));
-    const int nsub = (valid + kSubRows - 1) / kSubRows;
-    for (int sub = 0; sub < nsub; ++sub) {
-      const uint32_t slot = n % STAGES;
-      const uint32_t ph = (n / STAGES) & 1u;
-      if (!mbar_wait(smem_u32(&s.empty[slot]), ph ^ 1u, p.wait_limit_ns)) {
-        atomicOr(&g_sdq_dev_status, kDevTimeout);
-        ok = false;
-        break;
-      }
-      const uint32_t fb = smem_u32(&s.full[slot]);
-      mbar_arrive_expect_tx(fb, kStageBytes);
-      const uint32_t dst = smem_u32(s.ring[slot]);
-      const int r = static_cast<int>(row0) + sub * kSubRows;
-      tma_load_2d(dst, mx, fb, j * kG, r, pol);                               // gate
-      tma_load_2d(dst + kTensorStageBytes, mx, fb, p.K + j * kG, r, pol);     // up
-      tma_load_2d(dst + 2 * kTensorStageBytes, mg, fb, j * kG, r, pol);       // grad_y
-      ++n;
-    }
+// Round-half-even codes of a bf16 pair times `inv` (each half pre-multiplied
+// by `pre` first); each code is the low byte of its float's bits.
+template <bool kTiny>
+__device__ __forceinline__ float2 quant2(uint32_t v, float2 inv, float2 pre) {
+  float2 x = unpack2(v);
+  if (kTiny) x = __fmul2_rn(x, pre);
+  return __ffma2_rn(x, inv, make_float2(12582912.0f, 12582912.0f));
+}
+
+// Sixteen int8 codes of one row piece (8 bf16 pairs) with one inverse scale.
+template <bool kTiny>
+__device__ __forceinline__ uint4 quant16(const uint32_t (&v)[8], float inv) {
+  const float2 iv = make_float2(inv, inv);
+  const float2 pre = make_float2(kTinyPre, kTinyPre);
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 a = quant2<kTiny>(v[2 * k], iv, pre);
+    const float2 b = quant2<kTiny>(v[2 * k + 1], iv, pre);
+    w[k] = pack_low_bytes(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
+                          __float_as_uint(b.y));
   }
-  if (!ok) {
-    // Leave no copy in flight into this CTA's shared memory: the last load
-    // into each slot is the only one whose completion can still be pending.
-    const uint32_t first = n > STAGES ? n - STAGES : 0;
-    for (uint32_t k = first; k < n; ++k)
-      mbar_wait(smem_u32(&s.full[k % STAGES]), (k / STAGES) & 1u, p.wait_limit_ns);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Column pass: 16 tokens x 2 channels (one bf16 pair per token) -> two
+// 16-byte code rows (low channel, high channel).
+template <bool kTiny>
+__device__ __forceinline__ void quant_cols(const uint32_t (&v)[16], float2 inv, float2 pre,
+                                           uint4& lo, uint4& hi) {
+  uint32_t bl[16], bh[16];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const float2 q = quant2<kTiny>(v[t], inv, pre);
+    bl[t] = __float_as_uint(q.x);
+    bh[t] = __float_as_uint(q.y);
+  }
+  lo = make_uint4(pack_low_bytes(bl[0], bl[1], bl[2], bl[3]), pack_low_bytes(bl[4], bl[5], bl[6], bl[7]),
+                  pack_low_bytes(bl[8], bl[9], bl[10], bl[11]),
+                  pack_low_bytes(bl[12], bl[13], bl[14], bl[15]));
+  hi = make_uint4(pack_low_bytes(bh[0], bh[1], bh[2], bh[3]), pack_low_bytes(bh[4], bh[5], bh[6], bh[7]),
+                  pack_low_bytes(bh[8], bh[9], bh[10], bh[11]),
+                  pack_low_bytes(bh[12], bh[13], bh[14], bh[15]));
+}
+
+// 16 code bytes to a y_q_t row piece that may be cut short by the token count
+// or unaligned (M % 16 != 0).
+__device__ __forceinline__ void store_codes(int8_t* dst, uint4 o, int nb, bool vec16) {
+  if (vec16 && nb >= 16) {
+    *reinterpret_cast<uint4*>(dst) = o;
+    return;
+  }
+#pragma unroll
+  for (int b = 0; b < 16; ++b) {
+    const uint32_t w = b < 4 ? o.x : b < 8 ? o.y : b < 12 ? o.z : o.w;
+    if (b < nb) dst[b] = static_cast<int8_t>(w >> ((b & 3) * 8));
   }
 }
 
-template <int NW, int STAGES>
-__device__ __forceinline__ void consumer(Smem<NW, STAGES>& s, const Params& p, int warp,
-                                         int lane) {
-  using C = Config<NW, STAGES>;
-  constexpr int RPL = C::kRowsPerLane;          // token rows per lane per stage
-  constexpr int kRowsPerWarp = 2 * RPL;
+template <int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    fuse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy,
+                const Params p) {
   constexpr unsigned kFull = 0xffffffffu;
-  const int h = lane >> 4;                      // half-warp
-  const int q = lane & 15;                      // channels 8q .. 8q+7 of the tile
-  const int rho = (2 * warp + h) * RPL;         // first of this lane's rows in a stage
-  const int tid = threadIdx.x;                  // 0 .. kConsumers-1
+  extern __shared__ uint8_t smem_raw[];
+  auto& s = *reinterpret_cast<Smem<STAGES>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  // row pass: lane = 8 * rr + cq owns 16-byte chunks ca, cb (8 channels each)
+  // of row srow; the upper half of the row group takes them in swapped order
+  const int rr = lane >> 3;
+  const int cq = lane & 7;
+  const int ca = 2 * cq + (cq >> 2);
+  const int cb = 2 * cq + 1 - (cq >> 2);
+  const int srow = warp * kRowsPerWarp + rr;
+  // column pass: thread = 8 * cp + kc owns channels 2cp, 2cp+1 and tokens 16kc..16kc+15
+  const int cp = tid >> 3;
+  const int kc = tid & 7;
+  const int my_tiles = (p.num_tiles - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
+  const uint32_t total = static_cast<uint32_t>(my_tiles) * kStagesPerTile;
+  const uint64_t pol = l2_policy_evict_first();  // inputs are read exactly once
+
+  if (tid < 128) {
+    const float sc = __fdiv_rn(1.0f + static_cast<float>(tid) * (1.0f / 128.0f), 127.0f);
+    s.scale_tab[tid] = make_float2(sc, __frcp_rn(sc));
+  }
+  if (tid == 0) {
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_gy);
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(smem_u32(&s.full[st]), 1);
+      s.released[st] = 0;
+    }
+    fence_mbar_init();
+    const uint32_t first = total < STAGES ? total : STAGES;
+    s.issued = static_cast<int>(first);
+    for (uint32_t n = 0; n < first; ++n) issue_load(s, &map_x, &map_gy, p, n, pol);
+  }
+  __syncthreads();
+
   const int K = p.K;
   const int Kg = p.Kg;
   const int64_t M = p.M;
-  uint32_t n = 0;                               // stages consumed
+  const float2* tab = s.scale_tab;
   bool abort = false;
 
-  for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+  for (int k = 0; k < my_tiles; ++k) {
+    const int t = blockIdx.x + k * gridDim.x;
     int i, j;
     tile_ij(t, p.Mg, Kg, i, j);
     const int64_t row0 = int64_t(i) * kG;
-    const int valid = static_cast<int>((M - row0 < kG ? M - row0 : int64_t(kG)));
-    const int nsub = (valid + kSubRows - 1) / kSubRows;
+    const int valid = static_cast<int>(M - row0 < kG ? M - row0 : int64_t(kG));
+    uint8_t* yt = s.ytile[k & 1];
 
-    uint32_t yv[kNumSub][RPL][4];   // bf16 pairs of y, channels (8q+2k, 8q+2k+1)
-    uint32_t cmax[4] = {0u, 0u, 0u, 0u};
-
+    // ================= row pass over the tile's two stages
 #pragma unroll
-    for (int sub = 0; sub < kNumSub; ++sub) {
-#pragma unroll
-      for (int e = 0; e < RPL; ++e)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) yv[sub][e][k] = 0u;
-      if (sub >= nsub || abort) continue;
-
+    for (int sub = 0; sub < kStagesPerTile; ++sub) {
+      if (abort) continue;
+      const uint32_t n = static_cast<uint32_t>(k) * kStagesPerTile + sub;
       const uint32_t slot = n % STAGES;
-      const uint32_t ph = (n / STAGES) & 1u;
-      ++n;
-      const bool got = mbar_wait(smem_u32(&s.full[slot]), ph, p.wait_limit_ns);
+      const bool got = mbar_wait(smem_u32(&s.full[slot]), (n / STAGES) & 1u, p.wait_limit_ns);
       if (__any_sync(kFull, !got)) {
         abort = true;
         if (lane == 0) atomicOr(&g_sdq_dev_status, kDevTimeout);
         continue;
       }
 
-      // ---- stage -> registers, then hand the slot back to the producer
-      const uint8_t* st = s.ring[slot];
-      uint4 gv[RPL], uv[RPL], dv[RPL];
-#pragma unroll
-      for (int e = 0; e < RPL; ++e) {
-        const int off = (rho + e) * (kG * 2) + q * 16;
-        gv[e] = *reinterpret_cast<const uint4*>(st + off);
-        uv[e] = *reinterpret_cast<const uint4*>(st + kTensorStageBytes + off);
-        dv[e] = *reinterpret_cast<const uint4*>(st + 2 * kTensorStageBytes + off);
+      // ---- stage -> registers, then release the slot (the last warp refills it)
+      uint32_t gw[8], uw[8], dw[8];
+      {
+        const uint8_t* src = s.ring[slot] + srow * (kG * 2);
+        const uint4 g0 = *reinterpret_cast<const uint4*>(src + ca * 16);
+        const uint4 g1 = *reinterpret_cast<const uint4*>(src + cb * 16);
+        const uint4 u0 = *reinterpret_cast<const uint4*>(src + kBoxBytes + ca * 16);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(src + kBoxBytes + cb * 16);
+        const uint4 d0 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + ca * 16);
+        const uint4 d1 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + cb * 16);
+        gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
+        gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
+        uw[0] = u0.x; uw[1] = u0.y; uw[2] = u0.z; uw[3] = u0.w;
+        uw[4] = u1.x; uw[5] = u1.y; uw[6] = u1.z; uw[7] = u1.w;
+        dw[0] = d0.x; dw[1] = d0.y; dw[2] = d0.z; dw[3] = d0.w;
+        dw[4] = d1.x; dw[5] = d1.y; dw[6] = d1.z; dw[7] = d1.w;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&s.empty[slot]));
-
-      // ---- math, bf16 rounding, row amax of d_gate / d_up
-      uint32_t dgp[RPL][4], dup[RPL][4], P[RPL];
-#pragma unroll
-      for (int e = 0; e < RPL; ++e) {
-        const uint32_t* ga = reinterpret_cast<const uint32_t*>(&gv[e]);
-        const uint32_t* ua = reinterpret_cast<const uint32_t*>(&uv[e]);
-        const uint32_t* da = reinterpret_cast<const uint32_t*>(&dv[e]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          float y0, y1, g0, g1, u0, u1;
-          swiglu_bwd(bf16_lo(ga[k]), bf16_lo(ua[k]), bf16_lo(da[k]), y0, g0, u0);
-          swiglu_bwd(bf16_hi(ga[k]), bf16_hi(ua[k]), bf16_hi(da[k]), y1, g1, u1);
-          yv[sub][e][k] = pack_bf16x2(y0, y1);
-          dgp[e][k] = pack_bf16x2(g0, g1);
-          dup[e][k] = pack_bf16x2(u0, u1);
-          cmax[k] = absmax_bf16x2(cmax[k], yv[sub][e][k]);
-        }
-        const uint32_t a = absmax_bf16x2(absmax_bf16x2(dgp[e][0], dgp[e][1]),
-                                         absmax_bf16x2(dgp[e][2], dgp[e][3]));
-        const uint32_t b = absmax_bf16x2(absmax_bf16x2(dup[e][0], dup[e][1]),
-                                         absmax_bf16x2(dup[e][2], dup[e][3]));
-        // (hi half: d_gate, lo half: d_up)
-        uint32_t pr = absmax_bf16x2(__byte_perm(a, b, 0x1054), __byte_perm(a, b, 0x3276));
-#pragma unroll
-        for (int off = 1; off < 16; off <<= 1)
-          pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, off));
-        P[e] = pr & 0x7FFF7FFFu;
-      }
-
-      // ---- row scales: lane 2*rw + w computes (row rw of this warp, w = 0 d_gate / 1 d_up)
-      const int rw = (lane >> 1) & (kRowsPerWarp - 1);
-      const int src = (rw / RPL) << 4;
-      uint32_t psel = __shfl_sync(kFull, P[0], src);
-      if constexpr (RPL == 2) {
-        const uint32_t p1 = __shfl_sync(kFull, P[1], src);
-        psel = (rw & 1) ? p1 : psel;
-      }
-      const uint32_t abits = (lane & 1) ? (psel & 0xFFFFu) : (psel >> 16);
-      float scale, inv;
-      group_scale(__uint_as_float(abits << 16), scale, inv);
-      const int64_t srow0 = row0 + sub * kSubRows;
-      if (lane < 2 * kRowsPerWarp) {
-        const int64_t row = srow0 + 2 * warp * RPL + rw;
-        if (row < M) p.gis[row * (2 * Kg) + (lane & 1) * Kg + j] = scale;
-      }
-
-      // ---- quantize d_gate / d_up rows and store 8 bytes each
-#pragma unroll
-      for (int e = 0; e < RPL; ++e) {
-        const int sl = 2 * (h * RPL + e);
-        const float ig = __shfl_sync(kFull, inv, sl);
-        const float iu = __shfl_sync(kFull, inv, sl + 1);
-        const int64_t row = srow0 + rho + e;
-        if (row < M) {
-          uint2 og, ou;
-          og.x = pack_low_bytes(quant_bits(bf16_lo(dgp[e][0]), ig), quant_bits(bf16_hi(dgp[e][0]), ig),
-                                quant_bits(bf16_lo(dgp[e][1]), ig), quant_bits(bf16_hi(dgp[e][1]), ig));
-          og.y = pack_low_bytes(quant_bits(bf16_lo(dgp[e][2]), ig), quant_bits(bf16_hi(dgp[e][2]), ig),
-                                quant_bits(bf16_lo(dgp[e][3]), ig), quant_bits(bf16_hi(dgp[e][3]), ig));
-          ou.x = pack_low_bytes(quant_bits(bf16_lo(dup[e][0]), iu), quant_bits(bf16_hi(dup[e][0]), iu),
-                                quant_bits(bf16_lo(dup[e][1]), iu), quant_bits(bf16_hi(dup[e][1]), iu));
-          ou.y = pack_low_bytes(quant_bits(bf16_lo(dup[e][2]), iu), quant_bits(bf16_hi(dup[e][2]), iu),
-                                quant_bits(bf16_lo(dup[e][3]), iu), quant_bits(bf16_hi(dup[e][3]), iu));
-          int8_t* dst = p.giq + row * (2 * int64_t(K)) + j * kG + q * 8;
-          *reinterpret_cast<uint2*>(dst) = og;
-          *reinterpret_cast<uint2*>(dst + K) = ou;
-        }
-      }
-    }
-
-    // ---- tile end: column amax over the tile's tokens
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t c = cmax[k] & 0x7FFF7FFFu;
-      cmax[k] = absmax_bf16x2(c, __shfl_xor_sync(kFull, c, 16)) & 0x7FFF7FFFu;
-    }
-    if (h == 0)
-      *reinterpret_cast<uint4*>(&s.colmax[warp][q * 8]) = make_uint4(cmax[0], cmax[1], cmax[2], cmax[3]);
-    if (bar_red_or(1, C::kConsumers, abort)) break;  // every consumer stops together
-
-    if (tid < kG) {
-      uint32_t m = 0;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) m = max(m, static_cast<uint32_t>(s.colmax[w][tid]));
-      float scale, inv;
-      group_scale(__uint_as_float(m << 16), scale, inv);
-      p.yst[int64_t(j * kG + tid) * p.Mg + i] = scale;
-      s.inv_y[tid] = inv;
-    }
-    bar_sync(1, C::kConsumers);
-
-    // ---- quantize y and write it transposed into the staging tile
-    float iv[8];
-    *reinterpret_cast<float4*>(&iv[0]) = *reinterpret_cast<const float4*>(&s.inv_y[q * 8]);
-    *reinterpret_cast<float4*>(&iv[4]) = *reinterpret_cast<const float4*>(&s.inv_y[q * 8 + 4]);
-#pragma unroll
-    for (int sub = 0; sub < kNumSub; ++sub) {
-      const int tok = sub * kSubRows + rho;         // first token (within the tile) of this lane
-      const uint32_t word = static_cast<uint32_t>(tok >> 2) ^ static_cast<uint32_t>(q);
-      const uint32_t boff = (word << 2) + (tok & 3);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-          const int ch = q * 8 + 2 * k + hi;
-          const float inv = iv[2 * k + hi];
-          uint8_t* row = s.yt + ch * kG;
-          if constexpr (RPL == 2) {
-            const float v0 = hi ? bf16_hi(yv[sub][0][k]) : bf16_lo(yv[sub][0][k]);
-            const float v1 = hi ? bf16_hi(yv[sub][1][k]) : bf16_lo(yv[sub][1][k]);
-            const uint32_t b2 = __byte_perm(quant_bits(v0, inv), quant_bits(v1, inv), 0x0040);
-            *reinterpret_cast<uint16_t*>(row + boff) = static_cast<uint16_t>(b2);
-          } else {
-            const float v0 = hi ? bf16_hi(yv[sub][0][k]) : bf16_lo(yv[sub][0][k]);
-            row[boff] = static_cast<uint8_t>(quant_bits(v0, inv));
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&s.released[slot], 1) == kWarps - 1) {
+          __threadfence_block();
+          s.released[slot] = 0;
+          const uint32_t nn = n + STAGES;
+          if (nn < total) {
+            atomicMax(&s.issued, static_cast<int>(nn + 1));
+            issue_load(s, &map_x, &map_gy, p, nn, pol);
           }
         }
       }
-    }
-    bar_sync(1, C::kConsumers);
 
-    // ---- staging tile -> y_q_t: 16-token chunks, 8 lanes per 128-byte channel row
+      // ---- math, bf16 rounding; y to the shared tile (chunks swizzled by token)
+      uint32_t yv[8], dgp[8], dup[8];
 #pragma unroll
-    for (int it = 0; it < (kG * kG / 16) / C::kConsumers; ++it) {
-      const int idx = it * C::kConsumers + tid;
-      const int c = idx >> 3;
-      const int kc = idx & 7;
-      const uint32_t x = static_cast<uint32_t>(c >> 3);   // the row's swizzle key
-      const uint4 v = *reinterpret_cast<const uint4*>(s.yt + c * kG + ((kc ^ (x >> 2)) << 4));
-      // logical word m sits at word m ^ (x & 3) of the physical chunk
-      const bool s1 = x & 1u, s2 = x & 2u;
-      const uint32_t a0 = s1 ? v.y : v.x, a1 = s1 ? v.x : v.y;
-      const uint32_t a2 = s1 ? v.w : v.z, a3 = s1 ? v.z : v.w;
-      const uint4 o = make_uint4(s2 ? a2 : a0, s2 ? a3 : a1, s2 ? a0 : a2, s2 ? a1 : a3);
-      const int64_t tok = row0 + kc * 16;
-      if (tok < M) {
-        int8_t* dst = p.yqt + int64_t(j * kG + c) * M + tok;
-        if (p.yqt_vec16) {
-          *reinterpret_cast<uint4*>(dst) = o;
-        } else {
-          const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
-          const int nb = static_cast<int>((M - tok < 16 ? M - tok : int64_t(16)));
-          for (int b = 0; b < nb; ++b) dst[b] = static_cast<int8_t>(w4[b >> 2] >> ((b & 3) * 8));
-        }
+      for (int c = 0; c < 8; ++c) swiglu_bwd2(gw[c], uw[c], dw[c], yv[c], dgp[c], dup[c]);
+      {
+        const int tok = sub * kStageRows + srow;
+        const int key = (tok >> 4) & 7;
+        uint8_t* yrow = yt + tok * (kG * 2);
+        *reinterpret_cast<uint4*>(yrow + (ca ^ key) * 16) = make_uint4(yv[0], yv[1], yv[2], yv[3]);
+        *reinterpret_cast<uint4*>(yrow + (cb ^ key) * 16) = make_uint4(yv[4], yv[5], yv[6], yv[7]);
+      }
+
+      // ---- row amax of d_gate (hi half) and d_up (lo half) over the 8 lanes of the row
+      uint32_t a = absmax_bf16x2(dgp[0], dgp[1]), b = absmax_bf16x2(dup[0], dup[1]);
+#pragma unroll
+      for (int c = 2; c < 8; ++c) {
+        a = absmax_bf16x2(a, dgp[c]);
+        b = absmax_bf16x2(b, dup[c]);
+      }
+      uint32_t pr = absmax_bf16x2(__byte_perm(a, b, 0x1054), __byte_perm(a, b, 0x3276));
+      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 1));
+      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 2));
+      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 4));
+      pr &= 0x7FFF7FFFu;
+
+      // ---- the warp's 8 row scales: lane 2*r + w computes row r's d_gate (w = 0)
+      // or d_up (w = 1) scale, then every lane picks up its row's two
+      const int sr = (lane >> 1) & 3;
+      const uint32_t psel = __shfl_sync(kFull, pr, sr * 8);
+      float scale, inv;
+      group_scale((lane & 1) ? (psel & 0xFFFFu) : (psel >> 16), tab, scale, inv);
+      const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
+      if (lane < 8 && rbase + sr < valid)
+        p.gis[(row0 + rbase + sr) * (2 * Kg) + (lane & 1) * Kg + j] = scale;
+      const float ig = __shfl_sync(kFull, inv, 2 * rr);
+      const float iu = __shfl_sync(kFull, inv, 2 * rr + 1);
+
+      // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
+      const int r = rbase + rr;   // this lane's row within the tile
+      if (r < valid) {
+        const uint4 og = (ig < 0.0f) ? quant16<true>(dgp, -ig) : quant16<false>(dgp, ig);
+        const uint4 ou = (iu < 0.0f) ? quant16<true>(dup, -iu) : quant16<false>(dup, iu);
+        int8_t* dst = p.giq + (row0 + r) * (2 * int64_t(K)) + j * kG;
+        *reinterpret_cast<uint2*>(dst + ca * 8) = make_uint2(og.x, og.y);
+        *reinterpret_cast<uint2*>(dst + cb * 8) = make_uint2(og.z, og.w);
+        *reinterpret_cast<uint2*>(dst + K + ca * 8) = make_uint2(ou.x, ou.y);
+        *reinterpret_cast<uint2*>(dst + K + cb * 8) = make_uint2(ou.z, ou.w);
+      }
+    }
+
+    // every warp has written its y rows (and every warp agrees on stopping)
+    if (bar_red_or(1, kThreads, abort)) {
+      abort = true;
+      break;
+    }
+
+    // ================= column pass: channels 2cp, 2cp+1, tokens 16kc .. 16kc+15
+    {
+      uint32_t v[16];
+      const uint8_t* col = yt + (16 * kc) * (kG * 2) + ((cp ^ (4 * kc)) << 2);
+#pragma unroll
+      for (int tt = 0; tt < 16; ++tt) v[tt] = *reinterpret_cast<const uint32_t*>(col + tt * (kG * 2));
+      uint32_t m = absmax_bf16x2(v[0], v[1]);
+#pragma unroll
+      for (int tt = 2; tt < 16; ++tt) m = absmax_bf16x2(m, v[tt]);
+      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 1));
+      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 2));
+      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 4));
+      m &= 0x7FFF7FFFu;
+      float s_lo, i_lo, s_hi, i_hi;
+      group_scale(m & 0xFFFFu, tab, s_lo, i_lo);
+      group_scale(m >> 16, tab, s_hi, i_hi);
+      const int ch = j * kG + 2 * cp;
+      if (kc == 0) p.yst[int64_t(ch) * p.Mg + i] = s_lo;
+      if (kc == 1) p.yst[int64_t(ch + 1) * p.Mg + i] = s_hi;
+      uint4 lo, hi;
+      if (i_lo < 0.0f || i_hi < 0.0f) {
+        quant_cols<true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
+                         make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f),
+                         lo, hi);
+      } else {
+        quant_cols<false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
+      }
+      const int tok = 16 * kc;
+      if (tok < valid) {
+        const int nb = min(16, valid - tok);
+        int8_t* dst = p.yqt + int64_t(ch) * M + row0 + tok;
+        store_codes(dst, lo, nb, p.yqt_vec16 != 0);
+        store_codes(dst + M, hi, nb, p.yqt_vec16 != 0);
       }
     }
   }
-}
 
-template <int NW, int STAGES>
-__global__ void __launch_bounds__(Config<NW, STAGES>::kThreads, 1)
-    fuse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy,
-                const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  auto& s = *reinterpret_cast<Smem<NW, STAGES>*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < STAGES; ++st) {
-      mbar_init(smem_u32(&s.full[st]), 1);
-      mbar_init(smem_u32(&s.empty[st]), NW);
-    }
-    fence_mbar_init();
+  if (abort && tid == 0) {
+    // Leave no copy in flight into this CTA's shared memory: the last load
+    // issued into each slot is the only one whose completion can be pending.
+    const uint32_t issued = static_cast<uint32_t>(s.issued);
+    const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+    for (uint32_t n = first; n < issued; ++n)
+      mbar_wait(smem_u32(&s.full[n % STAGES]), (n / STAGES) & 1u, p.wait_limit_ns);
   }
-  __syncthreads();
-  if (warp == NW) {
-    if (lane == 0) producer<NW, STAGES>(s, &map_x, &map_gy, p);
-    return;
-  }
-  consumer<NW, STAGES>(s, p, warp, lane);
 }
 
 }  // namespace sdq

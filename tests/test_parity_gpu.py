@@ -197,3 +197,29 @@ def test_full_size_sampled_tiles_and_invariants(idx):
         st = U.compare(got, ref, f"{w.name} tile ({i},{j})")
         n_diff += st["grad_input_q"]["n_diff"] + st["y_q_t"]["n_diff"]
     _STATS[w.name + " (40 sampled tiles)"] = {"int8_n_diff": n_diff}
+
+
+def test_scales_exact_over_the_whole_exponent_range():
+    """Closed form, no oracle: gate = 32 makes sigma(32) round to 1 in fp32
+    (and silu(32), silu'(32) round to 32 and 1 in bf16 from fp64), so with
+    grad_y = 1 and up = a_i on every channel of token group i:
+        y = 32 a_i,  d_gate = a_i,  d_up = 32.
+    a_i sweeps one bf16 value per exponent field, subnormals included, so every
+    scale must equal the IEEE fp32 quotient amax / 127 and every code is 127."""
+    G = 128
+    pats = [0x0005, 0x0041, 0x007F] + [(e << 7) | ((e * 37) % 128) for e in range(1, 249)]
+    a = np.array(pats, dtype=np.uint16)
+    M, K = G * len(pats), 128
+    x = np.empty((M, 2 * K), np.uint16)
+    x[:, :K] = 0x4200                                   # 32.0
+    x[:, K:] = np.repeat(a, G)[:, None]
+    gy = np.full((M, K), 0x3F80, np.uint16)             # 1.0
+    giq, gis, yqt, yst = U.run_cuda(x, gy)
+    af = W.bf16_bits_to_f32(a)
+    f32 = np.float32
+    want_dg = af / f32(127)
+    want_y = (af * f32(32)) / f32(127)
+    assert np.array_equal(gis[:, 0], np.repeat(want_dg, G))
+    assert np.all(gis[:, 1] == f32(32) / f32(127))
+    assert np.array_equal(yst[0], want_y) and np.all(yst == yst[0:1])
+    assert np.all(giq == 127) and np.all(yqt == 127)
