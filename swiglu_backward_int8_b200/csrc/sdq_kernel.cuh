@@ -95,15 +95,24 @@ constexpr size_t smem_bytes() {
   return sizeof(Smem<STAGES>) + 128;  // + room to align the base to 128 B
 }
 
-// Tile t -> (token-group i, channel-group j), banded: 8 tile rows per band,
-// tile row fastest inside a band.
+// Tile t -> (token-group i, channel-group j), banded: kTileBand tile rows per
+// band, tile row fastest inside a band (a band of 1 is channel-group fastest).
+#ifndef SDQ_TILE_BAND
+#define SDQ_TILE_BAND 8
+#endif
 __device__ __forceinline__ void tile_ij(int t, int Mg, int Kg, int& i, int& j) {
-  constexpr int kBand = 8;
+  constexpr int kBand = SDQ_TILE_BAND;
+  static_assert(kBand > 0 && (kBand & (kBand - 1)) == 0, "band height must be a power of two");
   const int band = t / (kBand * Kg);
   const int r = t - band * (kBand * Kg);
   const int rows = min(kBand, Mg - band * kBand);
-  i = band * kBand + r % rows;
-  j = r / rows;
+  if (rows == kBand) {   // every band but the last: power-of-two height
+    i = band * kBand + (r & (kBand - 1));
+    j = r / kBand;
+  } else {
+    i = band * kBand + r % rows;
+    j = r / rows;
+  }
 }
 
 // Load n of this CTA: stage n % 2 of its (n / 2)-th tile, into slot n % STAGES.
@@ -132,10 +141,12 @@ __device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_
 // = silu*(1 - sigma) + sigma.  Results as bf16 pairs.
 __device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t dw, uint32_t& y,
                                             uint32_t& dg, uint32_t& du) {
+  constexpr float kNegLog2e = -1.4426950408889634f;  // e^-g = 2^(-g log2 e)
   const float2 g = unpack2(gw), u = unpack2(uw), dy = unpack2(dw);
   const float2 one = make_float2(1.0f, 1.0f);
-  const float2 d = __fadd2_rn(make_float2(__expf(-g.x), __expf(-g.y)), one);
-  const float2 sg = make_float2(__fdividef(1.0f, d.x), __fdividef(1.0f, d.y));  // 0 or 1 when saturated
+  const float2 xl = __fmul2_rn(g, make_float2(kNegLog2e, kNegLog2e));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(xl.x), ex2_approx(xl.y)), one);
+  const float2 sg = make_float2(rcp_approx(d.x), rcp_approx(d.y));  // 0 or 1 when saturated
   const float2 silu = __fmul2_rn(g, sg);
   const float2 oms = __ffma2_rn(sg, make_float2(-1.0f, -1.0f), one);
   const float2 dsilu = __ffma2_rn(silu, oms, sg);
@@ -160,6 +171,13 @@ __device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t d
 // same real number as v * fl(1/scale).
 constexpr float kTinyPre = 18446744073709551616.0f;  // 2^64
 
+// The rare branch, kept out of line so the common path stays short.
+__device__ __noinline__ float2 tiny_group_scale(uint32_t abits) {
+  if (abits == 0u) return make_float2(1.0f, 1.0f);
+  const float scale = __fdiv_rn(__uint_as_float(abits << 16), 127.0f);
+  return make_float2(scale, -__frcp_rn(scale * kTinyPre));
+}
+
 __device__ __forceinline__ void group_scale(uint32_t abits, const float2* tab, float& scale,
                                             float& inv_marked) {
   const uint32_t ex = abits >> 7;
@@ -168,12 +186,10 @@ __device__ __forceinline__ void group_scale(uint32_t abits, const float2* tab, f
     const int sh = (static_cast<int>(ex) - 127) << 23;
     scale = __int_as_float(__float_as_int(t.x) + sh);
     inv_marked = __int_as_float(__float_as_int(t.y) - sh);
-  } else if (abits != 0u) {
-    scale = __fdiv_rn(__uint_as_float(abits << 16), 127.0f);
-    inv_marked = -__frcp_rn(scale * kTinyPre);
   } else {
-    scale = 1.0f;
-    inv_marked = 1.0f;
+    const float2 r = tiny_group_scale(abits);
+    scale = r.x;
+    inv_marked = r.y;
   }
 }
 
@@ -377,8 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
       const int r = rbase + rr;   // this lane's row within the tile
       if (r < valid) {
-        const uint4 og = (ig < 0.0f) ? quant16<true>(dgp, -ig) : quant16<false>(dgp, ig);
-        const uint4 ou = (iu < 0.0f) ? quant16<true>(dup, -iu) : quant16<false>(dup, iu);
+        uint4 og, ou;
+        if (__any_sync(__activemask(), ig < 0.0f || iu < 0.0f)) {   // a tiny group in this warp (rare)
+          og = (ig < 0.0f) ? quant16<true>(dgp, -ig) : quant16<false>(dgp, ig);
+          ou = (iu < 0.0f) ? quant16<true>(dup, -iu) : quant16<false>(dup, iu);
+        } else {
+          og = quant16<false>(dgp, ig);
+          ou = quant16<false>(dup, iu);
+        }
         int8_t* dst = p.giq + (row0 + r) * (2 * int64_t(K)) + j * kG;
         *reinterpret_cast<uint2*>(dst + ca * 8) = make_uint2(og.x, og.y);
         *reinterpret_cast<uint2*>(dst + cb * 8) = make_uint2(og.z, og.w);
@@ -413,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kc == 0) p.yst[int64_t(ch) * p.Mg + i] = s_lo;
       if (kc == 1) p.yst[int64_t(ch + 1) * p.Mg + i] = s_hi;
       uint4 lo, hi;
-      if (i_lo < 0.0f || i_hi < 0.0f) {
+      if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
+        // pre-multiply only the tiny channels; the others use factor 1
         quant_cols<true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
                          make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f),
                          lo, hi);

@@ -116,6 +116,22 @@ __device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, bool 
   return r != 0;
 }
 
+// ---- special-function unit ----------------------------------------------------
+
+// 2^x, hardware approximation (relative error ~2^-22); subnormal results flush to 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 1/x, hardware approximation (within 1 ulp); 1/inf = 0, subnormal results flush to 0.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---- bf16 -------------------------------------------------------------------
 
 // Two fp32 -> packed bf16x2 (each rounded to nearest even); `lo` in bits 0..15.
