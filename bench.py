@@ -29,7 +29,6 @@ and the max-over-ranks of the timings.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import os
@@ -187,36 +186,6 @@ def dist_setup(args):
     return world, rank, local
 
 
-def dist_init(world, rank, local, backend="nccl"):
-    import torch
-    import torch.distributed as dist
-    if world > 1 and not dist.is_initialized():
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, rank=rank, world_size=world,
-                                timeout=datetime.timedelta(seconds=120),
-                                **({"device_id": torch.device("cuda", local)} if backend == "nccl" else {}))
-    return dist if world > 1 else None
-
-
-def max_over_ranks(value: float, dist, device) -> float:
-    if dist is None:
-        return value
-    import torch
-    t = torch.tensor([value], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def barrier(dist, device):
-    if dist is None:
-        return
-    import torch
-    t = torch.zeros(1, device=device)
-    dist.all_reduce(t)
-    torch.cuda.synchronize(device)
-
-
 # ---------------------------------------------------------------- CPU oracle timing
 
 def time_oracle(w: W.Workload, x, gy, min_seconds=10.0, max_rows=None):
@@ -289,7 +258,7 @@ def _to_device_bf16(a_u16, device):
     return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, dist):
+def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device):
     import torch
     import swiglu_backward_int8_b200 as sdq
     M, K = w.M, w.K
@@ -323,8 +292,9 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
                 call(warmup + done + k)
         graphs.append(g)
         done += n
+    from swiglu_backward_int8_b200 import parallel
     torch.cuda.synchronize(device)
-    barrier(dist, device)
+    parallel.barrier(device)
     torch.cuda.synchronize(device)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0 = time.time()
@@ -334,7 +304,7 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
     ev1.record(stream)
     torch.cuda.synchronize(device)
     t1 = time.time()
-    barrier(dist, device)
+    parallel.barrier(device)
     ms = ev0.elapsed_time(ev1)
     st = sdq.sdq_device_status(stream.cuda_stream)
     if st != 0:
@@ -373,10 +343,11 @@ def measure_e2e(w: W.Workload, x_np, gy_np, steps: int, device):
 def run_sdq(args):
     world, rank, local = dist_setup(args)
     import torch
-    dist = dist_init(world, rank, local)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     import swiglu_backward_int8_b200 as sdq  # fails loudly if the CUDA library is missing
+    from swiglu_backward_int8_b200 import parallel
+    parallel.init_from_env("nccl", timeout_s=120.0, device=device)
 
     w = pick_workload(args.workload)
     # Each rank its own replica (seed offset by rank): weak scaling, no exchange.
@@ -388,21 +359,21 @@ def run_sdq(args):
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     time.sleep(0.3)
-    ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, dist)
+    ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device)
     clocks = sampler.summary(t0, t1)
     sampler.stop()
-    ms_max = max_over_ranks(ms, dist, device)
+    ms_max = parallel.max_over_ranks(ms, device)
     per_step_ms = ms_max / args.steps
     bytes_step = w.algorithmic_bytes()
-    value = world * bytes_step * args.steps / (ms_max * 1e-3) / 1e9
+    value = parallel.aggregate_gbs(bytes_step * args.steps, world, ms_max)
     achieved = bytes_step / (per_step_ms * 1e-3) / 1e9
 
     e2e = None
     if not args.no_e2e:
         e2e_steps = args.e2e_steps or min(args.steps, 50)
         e = measure_e2e(wr, x_np, gy_np, e2e_steps, device)
-        e_ms = max_over_ranks(e["ms_per_step"], dist, device)
-        e["value"] = world * bytes_step / (e_ms * 1e-3) / 1e9
+        e_ms = parallel.max_over_ranks(e["ms_per_step"], device)
+        e["value"] = parallel.aggregate_gbs(bytes_step, world, e_ms)
         e2e = e
 
     per = None
@@ -411,8 +382,8 @@ def run_sdq(args):
         for ow in W.WORKLOADS:
             ox, og = W.make_inputs(ow)
             osteps = max(20, min(args.steps, int(2e9 // max(1, ow.algorithmic_bytes())) + 20))
-            oms, _, ons = measure_device(ow, ox, og, osteps, args.warmup, device, dist)
-            oms = max_over_ranks(oms, dist, device)
+            oms, _, ons = measure_device(ow, ox, og, osteps, args.warmup, device)
+            oms = parallel.max_over_ranks(oms, device)
             us = oms / osteps * 1e3
             gbs = ow.algorithmic_bytes() / (us * 1e-6) / 1e9
             per.append({"workload": ow.name, "M": ow.M, "K": ow.K, "us_per_call": us,
@@ -446,9 +417,10 @@ def run_sdq(args):
         if per is not None:
             line["per_workload"] = per
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        barrier(dist, device)
-        dist.destroy_process_group()
+    import torch.distributed as tdist
+    if tdist.is_initialized():
+        parallel.barrier(device)
+        tdist.destroy_process_group()
     return 0
 
 

@@ -160,6 +160,20 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
                           int64_t K, int32_t group_size, void* stream);
 
 /*
+ * sdq_fuse_test_stall -- test hook for the failure path, not for production
+ * use: sdq_fuse with the kernel's first shared-memory load withheld, so every
+ * CTA's first wait on its pipeline runs out after `wait_limit_ns`
+ * (1 us .. 1 s; outside that, SDQ_ERR_SHAPE).  The kernel then stops early,
+ * leaving its outputs incomplete, and the next sdq_device_status returns
+ * SDQ_ERR_TIMEOUT.  Nothing faults or hangs: every wait in the kernel is
+ * bounded, and the CUDA context stays usable for the next call.  (The page
+ * has no counterpart: it exists to test this library's failure detection.)
+ */
+int sdq_fuse_test_stall(const void* x, const void* grad_y, int8_t* grad_input_q,
+                        float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M,
+                        int64_t K, int32_t group_size, int64_t wait_limit_ns, void* stream);
+
+/*
  * sdq_device_status -- synchronizes `stream`, then reads and clears the
  * device-side status word of the current device: SDQ_OK, or
  * SDQ_ERR_TIMEOUT if a kernel's wait on its shared-memory pipeline ran past

@@ -34,6 +34,8 @@ _lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
 _lib.sdq_fuse_host_workspace_bytes.restype = ctypes.c_size_t
 _lib.sdq_fuse_host_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P]
 _lib.sdq_fuse_host_noalloc.restype = ctypes.c_int
+_lib.sdq_fuse_test_stall.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _I64, _P]
+_lib.sdq_fuse_test_stall.restype = ctypes.c_int
 _lib.sdq_device_status.argtypes = [_P]
 _lib.sdq_device_status.restype = ctypes.c_int
 _lib.sdq_status_string.argtypes = [ctypes.c_int]
@@ -116,6 +118,15 @@ def sdq_fuse_host_noalloc(x: int, grad_y: int, grad_input_q: int, grad_input_s: 
     ints; the outputs are complete once `stream` is synchronized."""
     _check(_lib.sdq_fuse_host_noalloc(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                                       group_size, stream or 0), "sdq_fuse_host_noalloc")
+
+
+def sdq_fuse_test_stall(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                        y_s_t: int, M: int, K: int, group_size: int, wait_limit_ns: int,
+                        stream: Optional[int] = None) -> None:
+    """Failure-path test hook: the kernel withholds its first load, so its
+    first bounded wait runs out; sdq_device_status then reports ERR_TIMEOUT."""
+    _check(_lib.sdq_fuse_test_stall(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                    group_size, wait_limit_ns, stream or 0), "sdq_fuse_test_stall")
 
 
 def sdq_fuse_host_workspace_bytes(M: int, K: int, chunk_rows: int = 0) -> int:

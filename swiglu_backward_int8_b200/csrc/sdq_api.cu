@@ -104,9 +104,10 @@ int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
   return SDQ_OK;
 }
 
-// Launch on validated arguments (M > 0).
+// Launch on validated arguments (M > 0).  `limit_ns` = 0: the default wait
+// limit; `withhold` = 1 only for the failure-path test hook.
 int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, float* yst,
-           int64_t M, int64_t K, cudaStream_t stream) {
+           int64_t M, int64_t K, cudaStream_t stream, uint64_t limit_ns = 0, int withhold = 0) {
   DeviceState* d = nullptr;
   int st = current_device(&d);
   if (st != SDQ_OK) return st;
@@ -124,7 +125,8 @@ int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, 
   p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
   p.num_tiles = p.Mg * p.Kg;
   p.yqt_vec16 = (M % 16 == 0) ? 1 : 0;
-  p.wait_limit_ns = wait_limit_ns();
+  p.wait_limit_ns = limit_ns ? limit_ns : wait_limit_ns();
+  p.withhold_first_load = withhold;
   const int grid = std::min(p.num_tiles, d->sms);
   sdq::fuse_kernel<kStages><<<grid, sdq::kThreads, sdq::smem_bytes<kStages>(), stream>>>(mx, mg, p);
   cudaError_t e = cudaGetLastError();
@@ -390,6 +392,16 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
       return cuda_fail(e);
   }
   return SDQ_OK;
+}
+
+int sdq_fuse_test_stall(const void* x, const void* grad_y, int8_t* grad_input_q,
+                        float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K,
+                        int32_t group_size, int64_t wait_limit_ns, void* stream) {
+  const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
+  if (st != SDQ_OK || M == 0) return st;
+  if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000) return SDQ_ERR_SHAPE;
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                static_cast<cudaStream_t>(stream), static_cast<uint64_t>(wait_limit_ns), 1);
 }
 
 int sdq_device_status(void* stream) {

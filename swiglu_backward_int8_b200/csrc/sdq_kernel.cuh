@@ -77,6 +77,7 @@ struct Params {
   int32_t Mg;
   int32_t num_tiles;
   int32_t yqt_vec16;  // M % 16 == 0: y_q_t rows take 16-byte stores
+  int32_t withhold_first_load;  // test hook: leave load 0 unissued so its wait runs out
   uint64_t wait_limit_ns;
 };
 
@@ -291,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     const uint32_t first = total < STAGES ? total : STAGES;
     s.issued = static_cast<int>(first);
-    for (uint32_t n = 0; n < first; ++n) issue_load(s, &map_x, &map_gy, p, n, pol);
+    for (uint32_t n = 0; n < first; ++n)
+      if (n != 0 || !p.withhold_first_load) issue_load(s, &map_x, &map_gy, p, n, pol);
   }
   __syncthreads();
 

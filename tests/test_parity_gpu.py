@@ -223,3 +223,23 @@ def test_scales_exact_over_the_whole_exponent_range():
     assert np.all(gis[:, 1] == f32(32) / f32(127))
     assert np.array_equal(yst[0], want_y) and np.all(yst == yst[0:1])
     assert np.all(giq == 127) and np.all(yqt == 127)
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """Failure detection without a fault: the test hook withholds the first
+    load, every CTA's first wait runs out after 20 ms, the kernel stops early,
+    the status word reports the timeout, and the next call is correct."""
+    import swiglu_backward_int8_b200 as sdq
+    from swiglu_backward_int8_b200 import _lib
+    w = W.small_workload(1024, 256, seed=31)
+    x, gy = W.make_inputs(w)
+    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
+    outs = sdq.allocate_outputs(w.M, w.K, "cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert sdq.sdq_device_status(stream) == sdq.Status.OK
+    _lib.sdq_fuse_test_stall(xd.data_ptr(), gyd.data_ptr(), *(o.data_ptr() for o in outs),
+                             w.M, w.K, 128, 20_000_000, stream)
+    assert sdq.sdq_device_status(stream) == sdq.Status.ERR_TIMEOUT
+    assert sdq.sdq_device_status(stream) == sdq.Status.OK      # read-and-clear
+    got = U.run_cuda(x, gy)                                     # the context is still usable
+    U.compare(got, oracle.silu_dot_fwd_bwd_quant_fuse(x, gy), "after a timeout")
