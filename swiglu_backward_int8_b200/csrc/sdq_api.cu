@@ -18,7 +18,7 @@ namespace {
 // Pipeline depth of the kernel's shared-memory ring (48 KB per stage;
 // compile-time overridable for tuning sweeps).
 #ifndef SDQ_STAGES
-#define SDQ_STAGES 3
+#define SDQ_STAGES 2
 #endif
 constexpr int kStages = SDQ_STAGES;
 

@@ -30,8 +30,10 @@
 //     once and shuffled back, quantization by multiplication with the inverse
 //     scale, coalesced stores; the bf16 y values go to a shared [token][channel]
 //     tile (double-buffered across tiles).
-//   * column pass, after one barrier per tile: a thread owns 2 channels x 16
-//     tokens of that tile, reduces the column amax over the 8 threads that
+//   * column pass, one tile late (after the row pass of the next tile, so no
+//     warp waits for the others at a tile boundary; two mbarriers per y buffer
+//     say "all rows written" and "all columns read"): a thread owns 2 channels
+//     x 16 tokens of the tile, reduces the column amax over the 8 threads that
 //     share its channels, computes the two column scales, quantizes its 32 y
 //     values and stores two 16-byte pieces of y_q_t rows; each group of 8
 //     threads writes one 128-byte line.
@@ -40,9 +42,9 @@
 //     opposite order, and the y tile's chunks are XOR-swizzled by token.
 //
 // Every wait on an mbarrier is bounded (Params::wait_limit_ns).  A wait that
-// runs out sets the device status word; the warps agree on stopping at the
-// next tile boundary through a barrier-reduction, and one thread waits
-// (bounded) for the copies still in flight before the CTA exits.
+// runs out sets the device status word and a shared abort flag that every
+// other wait polls, so all warps stop within one wait; after a final
+// __syncthreads one thread waits (bounded) for the copies still in flight.
 #pragma once
 
 #include <cstdint>
@@ -60,6 +62,10 @@ constexpr int kYBytes = kG * kG * 2;                // bf16 y tile: 32 KB
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerWarp = kStageRows / kWarps;   // 4 (8 lanes per row)
+#ifndef SDQ_YBUF
+#define SDQ_YBUF 2
+#endif
+constexpr int kYBuf = SDQ_YBUF;                     // y tiles in flight between row and column passes
 
 constexpr int kDevTimeout = 1;  // bit in the device status word
 
@@ -84,11 +90,14 @@ struct Params {
 template <int STAGES>
 struct Smem {
   alignas(128) uint8_t ring[STAGES][kStageBytes];  // [gate | up | grad_y], each [64][128] bf16
-  alignas(16) uint8_t ytile[2][kYBytes];           // bf16 y [token][channel], chunks swizzled
+  alignas(16) uint8_t ytile[kYBuf][kYBytes];       // bf16 y [token][channel], chunks swizzled
   alignas(16) float2 scale_tab[128];               // (fl((1+m/128)/127), 1/that) per bf16 mantissa m
   alignas(8) uint64_t full[STAGES];
+  alignas(8) uint64_t y_ready[kYBuf];              // all threads wrote their rows of the y tile
+  alignas(8) uint64_t y_free[kYBuf];               // all threads finished reading the y tile
   int released[STAGES];                            // warps done with the slot's current load
   int issued;                                      // loads issued so far (for the drain on abort)
+  int abort;                                       // set by the first wait that runs out
 };
 
 template <int STAGES>
@@ -243,13 +252,71 @@ __device__ __forceinline__ void quant_cols(const uint32_t (&v)[16], float2 inv, 
 // or unaligned (M % 16 != 0).
 __device__ __forceinline__ void store_codes(int8_t* dst, uint4 o, int nb, bool vec16) {
   if (vec16 && nb >= 16) {
-    *reinterpret_cast<uint4*>(dst) = o;
+    st_cs_v4(dst, o);
     return;
   }
 #pragma unroll
   for (int b = 0; b < 16; ++b) {
     const uint32_t w = b < 4 ? o.x : b < 8 ? o.y : b < 12 ? o.z : o.w;
     if (b < nb) dst[b] = static_cast<int8_t>(w >> ((b & 3) * 8));
+  }
+}
+
+// Bounded wait that also gives up as soon as another warp of the CTA has set
+// the abort flag; the first wait to run out sets the flag and the status word.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                              volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_sdq_dev_status, kDevTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Column pass of one tile: this thread's channels 2cp, 2cp+1 and tokens
+// 16kc .. 16kc+15 of the bf16 y tile -> column amax over the 8 threads that
+// share the channels, the two column scales, codes, two 16-byte pieces of
+// y_q_t rows.
+__device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab, const Params& p,
+                                            int i, int j, int64_t row0, int valid, int cp, int kc) {
+  constexpr unsigned kFull = 0xffffffffu;
+  uint32_t v[16];
+  const uint8_t* col = yt + (16 * kc) * (kG * 2) + ((cp ^ (4 * kc)) << 2);
+#pragma unroll
+  for (int tt = 0; tt < 16; ++tt) v[tt] = *reinterpret_cast<const uint32_t*>(col + tt * (kG * 2));
+  uint32_t m = absmax_bf16x2(v[0], v[1]);
+#pragma unroll
+  for (int tt = 2; tt < 16; ++tt) m = absmax_bf16x2(m, v[tt]);
+  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 1));
+  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 2));
+  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 4));
+  m &= 0x7FFF7FFFu;
+  float s_lo, i_lo, s_hi, i_hi;
+  group_scale(m & 0xFFFFu, tab, s_lo, i_lo);
+  group_scale(m >> 16, tab, s_hi, i_hi);
+  const int ch = j * kG + 2 * cp;
+  if (kc == 0) p.yst[int64_t(ch) * p.Mg + i] = s_lo;
+  if (kc == 1) p.yst[int64_t(ch + 1) * p.Mg + i] = s_hi;
+  uint4 lo, hi;
+  if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
+    // pre-multiply only the tiny channels; the others use factor 1
+    quant_cols<true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
+                     make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f), lo, hi);
+  } else {
+    quant_cols<false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
+  }
+  const int tok = 16 * kc;
+  if (tok < valid) {
+    const int nb = min(16, valid - tok);
+    int8_t* dst = p.yqt + int64_t(ch) * p.M + row0 + tok;
+    store_codes(dst, lo, nb, p.yqt_vec16 != 0);
+    store_codes(dst + p.M, hi, nb, p.yqt_vec16 != 0);
   }
 }
 
@@ -289,6 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&s.full[st]), 1);
       s.released[st] = 0;
     }
+    for (int b = 0; b < kYBuf; ++b) {
+      mbar_init(smem_u32(&s.y_ready[b]), kThreads);
+      mbar_init(smem_u32(&s.y_free[b]), kThreads);
+    }
+    s.abort = 0;
     fence_mbar_init();
     const uint32_t first = total < STAGES ? total : STAGES;
     s.issued = static_cast<int>(first);
@@ -301,28 +373,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Kg = p.Kg;
   const int64_t M = p.M;
   const float2* tab = s.scale_tab;
-  bool abort = false;
+  volatile int* abort_flag = &s.abort;
+  const uint64_t lim = p.wait_limit_ns;
+  bool ok = true;
+  // The column pass of tile k runs after the row pass of tile k+1, so warps
+  // never wait for each other at a tile boundary: y_ready[b] says every
+  // thread has written its rows of the tile in y buffer b, y_free[b] that
+  // every thread has read it; with kYBuf buffers a buffer is rewritten
+  // kYBuf tiles later, which leaves a warp slack.  Waits depend only on
+  // earlier points of the same per-warp sequence, so they cannot wait on
+  // each other in a cycle.
+  int pi = 0, pj = 0, pvalid = 0;   // the tile whose column pass is pending
+  int64_t prow0 = 0;
 
-  for (int k = 0; k < my_tiles; ++k) {
+  for (int k = 0; k < my_tiles && ok; ++k) {
     const int t = blockIdx.x + k * gridDim.x;
     int i, j;
     tile_ij(t, p.Mg, Kg, i, j);
     const int64_t row0 = int64_t(i) * kG;
     const int valid = static_cast<int>(M - row0 < kG ? M - row0 : int64_t(kG));
-    uint8_t* yt = s.ytile[k & 1];
+    const int yb = k % kYBuf;   // y buffer of this tile; tile t completes phase t / kYBuf of its barriers
+    uint8_t* yt = s.ytile[yb];
+    // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
+    int8_t* giq_t = p.giq + row0 * (2 * int64_t(K)) + j * kG;
+    float* gis_t = p.gis + row0 * (2 * Kg) + j;
 
     // ================= row pass over the tile's two stages
 #pragma unroll
     for (int sub = 0; sub < kStagesPerTile; ++sub) {
-      if (abort) continue;
       const uint32_t n = static_cast<uint32_t>(k) * kStagesPerTile + sub;
       const uint32_t slot = n % STAGES;
-      const bool got = mbar_wait(smem_u32(&s.full[slot]), (n / STAGES) & 1u, p.wait_limit_ns);
-      if (__any_sync(kFull, !got)) {
-        abort = true;
-        if (lane == 0) atomicOr(&g_sdq_dev_status, kDevTimeout);
-        continue;
-      }
+      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
+      if (!ok) break;
 
       // ---- stage -> registers, then release the slot (the last warp refills it)
       uint32_t gw[8], uw[8], dw[8];
@@ -355,10 +437,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- math, bf16 rounding; y to the shared tile (chunks swizzled by token)
+      // ---- math, bf16 rounding
       uint32_t yv[8], dgp[8], dup[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) swiglu_bwd2(gw[c], uw[c], dw[c], yv[c], dgp[c], dup[c]);
+
+      // ---- y to the shared tile (chunks swizzled by token); the buffer was
+      // last read by the column pass of tile k - kYBuf
+      if (sub == 0 && k >= kYBuf) {
+        ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_free[yb]), (k / kYBuf - 1) & 1, lim,
+                                             abort_flag));
+        if (!ok) break;
+      }
       {
         const int tok = sub * kStageRows + srow;
         const int key = (tok >> 4) & 7;
@@ -387,8 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float scale, inv;
       group_scale((lane & 1) ? (psel & 0xFFFFu) : (psel >> 16), tab, scale, inv);
       const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
-      if (lane < 8 && rbase + sr < valid)
-        p.gis[(row0 + rbase + sr) * (2 * Kg) + (lane & 1) * Kg + j] = scale;
+      if (lane < 8 && rbase + sr < valid) gis_t[(rbase + sr) * (2 * Kg) + (lane & 1) * Kg] = scale;
       const float ig = __shfl_sync(kFull, inv, 2 * rr);
       const float iu = __shfl_sync(kFull, inv, 2 * rr + 1);
 
@@ -403,65 +492,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           og = quant16<false>(dgp, ig);
           ou = quant16<false>(dup, iu);
         }
-        int8_t* dst = p.giq + (row0 + r) * (2 * int64_t(K)) + j * kG;
-        *reinterpret_cast<uint2*>(dst + ca * 8) = make_uint2(og.x, og.y);
-        *reinterpret_cast<uint2*>(dst + cb * 8) = make_uint2(og.z, og.w);
-        *reinterpret_cast<uint2*>(dst + K + ca * 8) = make_uint2(ou.x, ou.y);
-        *reinterpret_cast<uint2*>(dst + K + cb * 8) = make_uint2(ou.z, ou.w);
+        int8_t* dst = giq_t + r * (2 * K);
+        st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
+        st_cs_v2(dst + cb * 8, make_uint2(og.z, og.w));
+        st_cs_v2(dst + K + ca * 8, make_uint2(ou.x, ou.y));
+        st_cs_v2(dst + K + cb * 8, make_uint2(ou.z, ou.w));
       }
     }
+    if (!ok) break;
+    mbar_arrive(smem_u32(&s.y_ready[yb]));   // every thread: its y rows of tile k are written
 
-    // every warp has written its y rows (and every warp agrees on stopping)
-    if (bar_red_or(1, kThreads, abort)) {
-      abort = true;
-      break;
+    // ================= column pass of the previous tile
+    if (k >= 1) {
+      const int pb = (k - 1) % kYBuf;
+      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[pb]), ((k - 1) / kYBuf) & 1, lim,
+                                           abort_flag));
+      if (!ok) break;
+      column_pass(s.ytile[pb], tab, p, pi, pj, prow0, pvalid, cp, kc);
+      mbar_arrive(smem_u32(&s.y_free[pb]));
     }
-
-    // ================= column pass: channels 2cp, 2cp+1, tokens 16kc .. 16kc+15
-    {
-      uint32_t v[16];
-      const uint8_t* col = yt + (16 * kc) * (kG * 2) + ((cp ^ (4 * kc)) << 2);
-#pragma unroll
-      for (int tt = 0; tt < 16; ++tt) v[tt] = *reinterpret_cast<const uint32_t*>(col + tt * (kG * 2));
-      uint32_t m = absmax_bf16x2(v[0], v[1]);
-#pragma unroll
-      for (int tt = 2; tt < 16; ++tt) m = absmax_bf16x2(m, v[tt]);
-      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 1));
-      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 2));
-      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 4));
-      m &= 0x7FFF7FFFu;
-      float s_lo, i_lo, s_hi, i_hi;
-      group_scale(m & 0xFFFFu, tab, s_lo, i_lo);
-      group_scale(m >> 16, tab, s_hi, i_hi);
-      const int ch = j * kG + 2 * cp;
-      if (kc == 0) p.yst[int64_t(ch) * p.Mg + i] = s_lo;
-      if (kc == 1) p.yst[int64_t(ch + 1) * p.Mg + i] = s_hi;
-      uint4 lo, hi;
-      if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
-        // pre-multiply only the tiny channels; the others use factor 1
-        quant_cols<true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
-                         make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f),
-                         lo, hi);
-      } else {
-        quant_cols<false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
-      }
-      const int tok = 16 * kc;
-      if (tok < valid) {
-        const int nb = min(16, valid - tok);
-        int8_t* dst = p.yqt + int64_t(ch) * M + row0 + tok;
-        store_codes(dst, lo, nb, p.yqt_vec16 != 0);
-        store_codes(dst + M, hi, nb, p.yqt_vec16 != 0);
-      }
-    }
+    pi = i;
+    pj = j;
+    prow0 = row0;
+    pvalid = valid;
   }
 
-  if (abort && tid == 0) {
+  // column pass of the last tile
+  if (ok && my_tiles > 0) {
+    const int k = my_tiles - 1;
+    ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[k % kYBuf]), (k / kYBuf) & 1, lim,
+                                         abort_flag));
+    if (ok) column_pass(s.ytile[k % kYBuf], tab, p, pi, pj, prow0, pvalid, cp, kc);
+  }
+
+  __syncthreads();   // every thread arrives here, whether it stopped early or not
+  if (tid == 0 && *abort_flag) {
     // Leave no copy in flight into this CTA's shared memory: the last load
     // issued into each slot is the only one whose completion can be pending.
     const uint32_t issued = static_cast<uint32_t>(s.issued);
     const uint32_t first = issued > STAGES ? issued - STAGES : 0;
     for (uint32_t n = first; n < issued; ++n)
-      mbar_wait(smem_u32(&s.full[n % STAGES]), (n / STAGES) & 1u, p.wait_limit_ns);
+      mbar_wait(smem_u32(&s.full[n % STAGES]), (n / STAGES) & 1u, lim);
   }
 }
 

@@ -96,6 +96,20 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ---- streaming stores ---------------------------------------------------------
+// Output codes are written once and not read again by this kernel: stores with
+// the evict-first (.cs) policy keep them from displacing other lines in L2.
+
+__device__ __forceinline__ void st_cs_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_cs_v2(void* p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
 // ---- named barriers ---------------------------------------------------------
 
 __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t nthreads) {
