@@ -470,16 +470,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 4));
       pr &= 0x7FFF7FFFu;
 
-      // ---- the warp's 8 row scales: lane 2*r + w computes row r's d_gate (w = 0)
-      // or d_up (w = 1) scale, then every lane picks up its row's two
-      const int sr = (lane >> 1) & 3;
-      const uint32_t psel = __shfl_sync(kFull, pr, sr * 8);
-      float scale, inv;
-      group_scale((lane & 1) ? (psel & 0xFFFFu) : (psel >> 16), tab, scale, inv);
+      // ---- the row's two scales, computed by each of its 8 lanes (no shuffles
+      // on this path); lanes 0 and 1 of the row store them
+      float sg, ig, su, iu;
+      group_scale(pr >> 16, tab, sg, ig);
+      group_scale(pr & 0xFFFFu, tab, su, iu);
       const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
-      if (lane < 8 && rbase + sr < valid) gis_t[(rbase + sr) * (2 * Kg) + (lane & 1) * Kg] = scale;
-      const float ig = __shfl_sync(kFull, inv, 2 * rr);
-      const float iu = __shfl_sync(kFull, inv, 2 * rr + 1);
+      if (cq < 2 && rbase + rr < valid) gis_t[(rbase + rr) * (2 * Kg) + cq * Kg] = cq ? su : sg;
 
       // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
       const int r = rbase + rr;   // this lane's row within the tile
