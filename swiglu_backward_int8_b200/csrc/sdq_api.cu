@@ -128,8 +128,22 @@ int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, 
   p.wait_limit_ns = limit_ns ? limit_ns : wait_limit_ns();
   p.withhold_first_load = withhold;
   const int grid = std::min(p.num_tiles, d->sms);
-  sdq::fuse_kernel<kStages><<<grid, sdq::kThreads, sdq::smem_bytes<kStages>(), stream>>>(mx, mg, p);
-  cudaError_t e = cudaGetLastError();
+  // Programmatic stream serialization: this launch may begin while the
+  // previous kernel of the stream drains; the kernel's griddepcontrol.wait
+  // keeps every global access behind that kernel's completion.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(sdq::kThreads);
+  cfg.dynamicSmemBytes = sdq::smem_bytes<kStages>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, sdq::fuse_kernel<kStages>, mx, mg, p);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return SDQ_OK;
 }

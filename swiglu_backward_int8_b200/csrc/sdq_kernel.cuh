@@ -362,11 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     s.abort = 0;
     fence_mbar_init();
+    grid_dependency_wait();   // inputs may come from the previous kernel in the stream
     const uint32_t first = total < STAGES ? total : STAGES;
     s.issued = static_cast<int>(first);
     for (uint32_t n = 0; n < first; ++n)
       if (n != 0 || !p.withhold_first_load) issue_load(s, &map_x, &map_gy, p, n, pol);
   }
+  grid_dependency_wait();   // every thread: global memory only after the previous grid is done
+  grid_launch_dependents();
   __syncthreads();
 
   const int K = p.K;

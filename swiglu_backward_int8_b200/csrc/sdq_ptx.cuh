@@ -110,6 +110,21 @@ __device__ __forceinline__ void st_cs_v2(void* p, uint2 v) {
   asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+
+// Waits until the grids this one depends on (the previous kernel in the
+// stream, under programmatic stream serialization) have completed and their
+// memory operations are visible; returns at once without such a dependency.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel in the stream start launching its CTAs (it still
+// waits for this grid to complete before touching memory).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- named barriers ---------------------------------------------------------
 
 __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t nthreads) {
