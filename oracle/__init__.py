@@ -60,6 +60,19 @@ def lib() -> ctypes.CDLL:
         L.oracle_swiglu_bwd_bf16.restype = None
         L.oracle_silu_dot_fwd_bwd_quant_fuse.argtypes = [P, P, P, P, P, P, i64, i64, i64]
         L.oracle_silu_dot_fwd_bwd_quant_fuse.restype = ctypes.c_int
+        L.oracle_e4m3_rne.argtypes = [dbl]
+        L.oracle_e4m3_rne.restype = ctypes.c_uint8
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = dbl
+        L.oracle_e8m0_ceil.argtypes = [ctypes.c_float]
+        L.oracle_e8m0_ceil.restype = ctypes.c_uint8
+        L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_value.restype = dbl
+        L.oracle_quant_group_fmt.argtypes = [P, i64, i64, P, i64, P, ctypes.c_int, ctypes.c_int]
+        L.oracle_quant_group_fmt.restype = None
+        L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.argtypes = [P, P, P, P, P, P, i64, i64, i64,
+                                                             ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -137,4 +150,76 @@ def silu_dot_fwd_bwd_quant_fuse(x: np.ndarray, grad_y: np.ndarray, group_size: i
                                                   _ptr(yqt), _ptr(yst), M, K, G)
     if rc != 0:
         raise ValueError(f"oracle rejected M={M} K={K} group_size={G}")
+    return giq, gis, yqt, yst
+
+
+# ---- output formats (codes: 0 INT8, 1 E4M3; scales: 0 fp32, 1 E8M0;
+# ys_layout: 0 y_s_t [K, Mg], 1 [Mg, K]) -------------------------------------
+
+CODES_INT8, CODES_E4M3 = 0, 1
+SCALES_FP32, SCALES_E8M0 = 0, 1
+YS_K_MG, YS_MG_K = 0, 1
+
+
+def e4m3_rne(v: float) -> int:
+    """Nearest OCP E4M3 code (byte) of a double, ties to even, saturating at 448."""
+    return int(lib().oracle_e4m3_rne(float(v)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().oracle_e4m3_value(int(code)))
+
+
+def e8m0_ceil(s: float) -> int:
+    """E8M0 byte of the smallest power of two >= s (s a positive float32)."""
+    return int(lib().oracle_e8m0_ceil(float(s)))
+
+
+def e8m0_value(e: int) -> float:
+    return float(lib().oracle_e8m0_value(int(e)))
+
+
+def quant_group_fmt(v_bf16: np.ndarray, codes: int = 0, scales: int = 0):
+    """One group of bf16 bit patterns -> (code bytes uint8, scale) where the
+    scale is a float (fp32 scales) or an int byte (E8M0)."""
+    v = np.ascontiguousarray(v_bf16, dtype=np.uint16)
+    q = np.zeros(v.size, dtype=np.uint8)
+    s = np.zeros(4, dtype=np.uint8)
+    lib().oracle_quant_group_fmt(_ptr(v), v.size, 1, _ptr(q), 1, _ptr(s), int(codes), int(scales))
+    return q, (int(s[0]) if scales else float(s.view(np.float32)[0]))
+
+
+def output_shapes_fmt(M: int, K: int, group_size: int = 128, ys_layout: int = 0):
+    G = int(group_size)
+    Kg, Mg = K // G, (M + G - 1) // G
+    return (M, 2 * K), (M, 2 * Kg), (K, M), ((Mg, K) if ys_layout else (K, Mg))
+
+
+def silu_dot_fwd_bwd_quant_fuse_fmt(x: np.ndarray, grad_y: np.ndarray, group_size: int = 128,
+                                    codes: int = 0, scales: int = 0, ys_layout: int = 0):
+    """The whole op in a chosen output format, on uint16 (bf16 bit) arrays.
+
+    Returns ``(grad_input_q [M,2K] uint8 code bytes, grad_input_s [M,2K/G],
+    y_q_t [K,M] uint8, y_s_t [K,Mg] or [Mg,K])``; scale arrays are float32
+    (fp32 scales) or uint8 (E8M0 bytes).
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    gy = np.ascontiguousarray(grad_y, dtype=np.uint16)
+    M, K = gy.shape
+    assert x.shape == (M, 2 * K), (x.shape, gy.shape)
+    G = int(group_size)
+    if G < 1 or K % G:
+        raise ValueError(f"K={K} is not a multiple of group_size={G}")
+    sq, ss, yq, ys = output_shapes_fmt(M, K, G, ys_layout)
+    sdt = np.uint8 if scales else np.float32
+    giq = np.zeros(sq, np.uint8)
+    gis = np.zeros(ss, sdt)
+    yqt = np.zeros(yq, np.uint8)
+    yst = np.zeros(ys, sdt)
+    rc = lib().oracle_silu_dot_fwd_bwd_quant_fuse_fmt(_ptr(x), _ptr(gy), _ptr(giq), _ptr(gis),
+                                                      _ptr(yqt), _ptr(yst), M, K, G,
+                                                      int(codes), int(scales), int(ys_layout))
+    if rc != 0:
+        raise ValueError(f"oracle rejected M={M} K={K} group_size={G} format "
+                         f"({codes}, {scales}, {ys_layout})")
     return giq, gis, yqt, yst

@@ -40,6 +40,30 @@
 //   whole op               closed-form hand-derived cases (gate = 0, gate
 //                          large), layout/transposition patterns, tail and
 //                          zero groups, and a hand-derived golden fixture.
+//
+// Output formats beyond the page's (INT8 codes, fp32 scales, y_s_t [K, Mg]);
+// the page only says the outputs feed quantized GEMMs, so these follow public
+// format definitions, each reading listed in the design notes:
+//   * FP8 codes: OCP 8-bit floating point, E4M3 variant (sign, 4 exponent
+//     bits with bias 7, 3 mantissa bits; no infinities; S.1111.111 is NaN, so
+//     the largest finite magnitude is 448).  scale = fl32(amax / 448); a code
+//     is the nearest E4M3 value of the fp32 quotient v / scale, ties to an
+//     even mantissa, magnitudes above 448 saturated to 448.
+//   * E8M0 scales: OCP Microscaling (MX) scale format, an unsigned biased
+//     exponent byte e with value 2^(e - 127).  The scale is the smallest
+//     power of two not below fl32(amax / Qmax) (Qmax = 127 for INT8 codes,
+//     448 for E4M3), so no element exceeds the code range, clamped to
+//     [2^-127, 2^127]; an all-zero group gets 2^0 (byte 127).
+//   * y_s_t [Mg, K]: token group i, channel k at i * K + k.
+// Pins (tests/test_oracle_formats.py): oracle_e4m3_rne against torch's
+// float8_e4m3fn conversion inside the finite range and against brute force
+// over all 127 finite magnitudes with exact rationals; oracle_e8m0_ceil
+// against brute force over the 255 powers of two; oracle_quant_group_fmt
+// against exact-rational brute force of each definition and its invariants
+// (scale/2 < amax/Qmax <= scale, |code| <= Qmax, the amax element reaches
+// the top binade); the whole op against the pinned INT8 whole op (default
+// format), a transposition identity between the two y_s_t layouts, and
+// closed-form cases.
 
 #include <cmath>
 #include <cstdint>
@@ -180,6 +204,126 @@ int oracle_silu_dot_fwd_bwd_quant_fuse(const uint16_t* x, const uint16_t* grad_y
       const int64_t n = (M - t0 < G) ? (M - t0) : G;
       oracle_quant_group(&y[t0 * K + k], n, K, &y_q_t[k * M + t0], 1,
                          &y_s_t[k * Mg + i]);
+    }
+  }
+  return 0;
+}
+
+// ---- output formats ---------------------------------------------------------
+
+// Nearest OCP E4M3 code of a double, ties to an even mantissa, in one rounding
+// step; magnitudes above 448 saturate to 448 (code 0x7E); NaN gives 0x7F.
+uint8_t oracle_e4m3_rne(double v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(v);
+  if (a > 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int e = std::ilogb(a);            // 2^e <= a < 2^(e+1)
+  if (e < -6) e = -6;               // below the normal range the spacing stays 2^-9
+  const double ulp = std::ldexp(1.0, e - 3);
+  const double r = std::nearbyint(a / ulp) * ulp;  // a/ulp is exact; nearbyint ties to even
+  if (r < std::ldexp(1.0, -6))      // subnormal: exponent field 0, mantissa r / 2^-9
+    return sign | static_cast<uint8_t>(r / std::ldexp(1.0, -9));
+  const int re = std::ilogb(r);     // r may have rounded up into the next binade
+  const int mant = static_cast<int>(r / std::ldexp(1.0, re - 3)) - 8;
+  return sign | static_cast<uint8_t>(((re + 7) << 3) | mant);
+}
+
+// Value of an E4M3 code (NaN for S.1111.111).
+double oracle_e4m3_value(uint8_t c) {
+  const double sign = (c & 0x80) ? -1.0 : 1.0;
+  const int ef = (c >> 3) & 0xF;
+  const int mf = c & 0x7;
+  if (ef == 0xF && mf == 0x7) return std::nan("");
+  if (ef == 0) return sign * std::ldexp(static_cast<double>(mf), -9);
+  return sign * std::ldexp(1.0 + mf / 8.0, ef - 7);
+}
+
+// E8M0 byte of the smallest power of two >= s (s > 0), clamped to
+// [2^-127, 2^127]: value 2^(e - 127).
+uint8_t oracle_e8m0_ceil(float s) {
+  const double d = static_cast<double>(s);
+  int k = std::ilogb(d);                    // 2^k <= d < 2^(k+1)
+  if (std::ldexp(1.0, k) < d) k += 1;       // not a power of two: round up
+  if (k < -127) k = -127;
+  if (k > 127) k = 127;
+  return static_cast<uint8_t>(k + 127);
+}
+
+double oracle_e8m0_value(uint8_t e) { return std::ldexp(1.0, static_cast<int>(e) - 127); }
+
+// Quantize one group of n bf16 values (element i at v[i*stride]) in a chosen
+// format.  codes: 0 INT8 (q as int8 bits), 1 E4M3; scales: 0 fp32 (*scale is
+// a float), 1 E8M0 (*scale is one byte).  All-zero group: codes 0, scale 1.
+void oracle_quant_group_fmt(const uint16_t* v, int64_t n, int64_t stride, uint8_t* q,
+                            int64_t qstride, void* scale, int codes, int scales) {
+  const float qmax = codes ? 448.0f : 127.0f;
+  float amax = 0.0f;
+  for (int64_t i = 0; i < n; ++i) {
+    const float a = std::fabs(bf16_to_float(v[i * stride]));
+    if (a > amax) amax = a;
+  }
+  double s;   // the scale's value
+  if (amax == 0.0f) {
+    s = 1.0;
+  } else {
+    const float s32 = amax / qmax;   // fp32 division, rounded once
+    s = scales ? oracle_e8m0_value(oracle_e8m0_ceil(s32)) : static_cast<double>(s32);
+  }
+  if (scales) *static_cast<uint8_t*>(scale) = oracle_e8m0_ceil(static_cast<float>(s));
+  else *static_cast<float*>(scale) = static_cast<float>(s);
+  for (int64_t i = 0; i < n; ++i) {
+    uint8_t c = 0;
+    if (amax != 0.0f) {
+      // the quotient rounded once to fp32 (exact for a power-of-two scale)
+      const float t = static_cast<float>(static_cast<double>(bf16_to_float(v[i * stride])) / s);
+      if (codes) {
+        c = oracle_e4m3_rne(t);
+      } else {
+        float r = std::nearbyint(t);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        c = static_cast<uint8_t>(static_cast<int8_t>(r));
+      }
+    }
+    q[i * qstride] = c;
+  }
+}
+
+// The whole op in a chosen format.  codes / scales as in
+// oracle_quant_group_fmt; ys_layout: 0 y_s_t [K, Mg], 1 [Mg, K].  Code
+// arrays are bytes; scale arrays are fp32 or one byte per scale.
+int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* grad_y,
+                                           uint8_t* grad_input_q, void* grad_input_s,
+                                           uint8_t* y_q_t, void* y_s_t, int64_t M, int64_t K,
+                                           int64_t group_size, int codes, int scales,
+                                           int ys_layout) {
+  const int64_t G = group_size;
+  if (G < 1 || M < 0 || K < 0 || K % G != 0) return -1;
+  if (codes < 0 || codes > 1 || scales < 0 || scales > 1 || ys_layout < 0 || ys_layout > 1) return -1;
+  if (M == 0 || K == 0) return 0;
+  const int64_t Kg = K / G;
+  const int64_t Mg = (M + G - 1) / G;
+  const int64_t sb = scales ? 1 : 4;   // bytes per scale
+  uint8_t* gis = static_cast<uint8_t*>(grad_input_s);
+  uint8_t* yst = static_cast<uint8_t*>(y_s_t);
+  std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
+  oracle_swiglu_bwd_bf16(x, grad_y, M, K, y.data(), dg.data(), du.data());
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t j = 0; j < 2 * Kg; ++j) {
+      const uint16_t* src = (j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G];
+      oracle_quant_group_fmt(src, G, 1, &grad_input_q[m * 2 * K + j * G], 1,
+                             gis + (m * 2 * Kg + j) * sb, codes, scales);
+    }
+  }
+  for (int64_t k = 0; k < K; ++k) {
+    for (int64_t i = 0; i < Mg; ++i) {
+      const int64_t t0 = i * G;
+      const int64_t n = (M - t0 < G) ? (M - t0) : G;
+      const int64_t si = ys_layout ? (i * K + k) : (k * Mg + i);
+      oracle_quant_group_fmt(&y[t0 * K + k], n, K, &y_q_t[k * M + t0], 1, yst + si * sb, codes,
+                             scales);
     }
   }
   return 0;

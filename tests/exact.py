@@ -80,3 +80,67 @@ def f64_to_bf16_bits(vals) -> np.ndarray:
     bits = f.view(np.uint32)
     assert np.all((bits & np.uint32(0xFFFF)) == 0), "value is not a bf16"
     return (bits >> np.uint32(16)).astype(np.uint16)
+
+
+# ---- formats beyond bf16 (exact rationals; nothing here calls the oracle) ----
+
+def round_half_even(v: Fraction) -> int:
+    """Nearest integer to an exact rational, ties to the even integer."""
+    fl = v.numerator // v.denominator
+    rem = v - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        return fl + 1
+    return fl
+
+
+def _floor_log2(a: Fraction) -> int:
+    """k with 2^k <= a < 2^(k+1), for a > 0."""
+    k = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** k > a:
+        k -= 1
+    while Fraction(2) ** (k + 1) <= a:
+        k += 1
+    return k
+
+
+def f32_round(v: Fraction) -> Fraction:
+    """Float32 nearest to an exact rational (ties to even, subnormals kept,
+    no overflow handling: callers stay inside the finite range)."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = max(_floor_log2(a), -126)
+    ulp = Fraction(2) ** (e - 23)
+    return sign * round_half_even(a / ulp) * ulp
+
+
+def e4m3_table():
+    """(value, code) of the 127 non-negative finite OCP E4M3 codes 0x00..0x7E:
+    exponent field 0 holds m * 2^-9, field f > 0 holds (1 + m/8) * 2^(f-7)."""
+    out = []
+    for code in range(0x7F):
+        f, m = code >> 3, code & 7
+        val = Fraction(m, 2 ** 9) if f == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (f - 7)
+        out.append((val, code))
+    return out
+
+
+_E4M3 = e4m3_table()
+
+
+def e4m3_nearest(v: Fraction) -> int:
+    """E4M3 code nearest to v by exhaustive comparison (ties to the even code,
+    magnitudes above 448 saturate to 448)."""
+    sign = 0x80 if v < 0 else 0
+    a = abs(v)
+    if a > 448:
+        return sign | 0x7E
+    best = min(_E4M3, key=lambda vc: (abs(vc[0] - a), vc[1] & 1))
+    return sign | best[1]
+
+
+def pow2_ceil_exponent(v: Fraction) -> int:
+    """Smallest k with 2^k >= v (v > 0)."""
+    k = _floor_log2(v)
+    return k if Fraction(2) ** k == v else k + 1

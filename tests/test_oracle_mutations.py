@@ -33,10 +33,33 @@ MUTATIONS = [
     ("if (e < -126) e = -126;", "", "test_bf16_rne_against_torch_float32_conversion"),
     ("return 1.0 / (1.0 + std::exp(-g));", "return 1.0 / (1.0 + std::exp(-(float)g));",
      "test_sigmoid_matches_library_expit"),
+    # output formats (pins in test_oracle_formats.py)
+    ("if (e < -6) e = -6;", "", "test_e4m3_rne_bruteforce_exact_rationals", "formats"),
+    ("std::ldexp(1.0, e - 3)", "std::ldexp(1.0, e - 4)", "test_e4m3_rne_against_torch_float8_conversion",
+     "formats"),
+    ("const double r = std::nearbyint(a / ulp) * ulp;  // a/ulp is exact; nearbyint ties to even\n"
+     "  if (r < std::ldexp(1.0, -6))",
+     "const double r = std::round(a / ulp) * ulp;\n  if (r < std::ldexp(1.0, -6))",
+     "test_e4m3_rne_bruteforce_exact_rationals", "formats"),
+    ("if (a > 448.0) return sign | 0x7E;", "if (a > 480.0) return sign | 0x7E;",
+     "test_e4m3_rne_bruteforce_exact_rationals", "formats"),
+    ("if (std::ldexp(1.0, k) < d) k += 1;", "", "test_e8m0_ceil_bruteforce", "formats"),
+    ("if (k < -127) k = -127;", "", "test_e8m0_ceil_bruteforce", "formats"),
+    ("const float qmax = codes ? 448.0f : 127.0f;", "const float qmax = codes ? 447.0f : 127.0f;",
+     "test_quant_group_fmt_bruteforce", "formats"),
+    ("s = scales ? oracle_e8m0_value(oracle_e8m0_ceil(s32)) : static_cast<double>(s32);",
+     "s = static_cast<double>(s32);", "test_quant_group_fmt_bruteforce", "formats"),
+    ("const int64_t si = ys_layout ? (i * K + k) : (k * Mg + i);",
+     "const int64_t si = ys_layout ? (k * Mg + i) : (k * Mg + i);",
+     "test_whole_op_fmt_ys_layouts_transpose", "formats"),
+    ("oracle_quant_group_fmt(&y[t0 * K + k], n, K,", "oracle_quant_group_fmt(&y[t0 * K + k], n, 1,",
+     "test_whole_op_fmt_groups_relate_to_stage1", "formats"),
 ]
 
+PIN_FILES = {"pins": "test_oracle_pins.py", "formats": "test_oracle_formats.py"}
 
-def _run_mutant(tmp_dir, idx, old, new, pin):
+
+def _run_mutant(tmp_dir, idx, old, new, pin, pins="pins"):
     src = open(oracle._SRC).read()
     if src.count(old) < 1:
         return f"mutation #{idx} no longer applies: {old!r}"
@@ -47,7 +70,7 @@ def _run_mutant(tmp_dir, idx, old, new, pin):
     subprocess.run(["g++", *oracle.CXXFLAGS, mutated, "-o", so], check=True)
     env = dict(os.environ, SDQ_ORACLE_LIB=so)
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", pin],
+                        os.path.join(ROOT, "tests", PIN_FILES[pins]), "-k", pin],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     if r.returncode == 0:
         return f"planted mistake #{idx} survived {pin}: {old!r} -> {new!r}"
