@@ -54,6 +54,8 @@
 //     power of two not below fl32(amax / Qmax) (Qmax = 127 for INT8 codes,
 //     448 for E4M3), so no element exceeds the code range, clamped to
 //     [2^-127, 2^127]; an all-zero group gets 2^0 (byte 127).
+//   * In every format an all-zero group has scale 1 and each code is that of
+//     v / 1: zero, with v's sign in E4M3 (0x80 for -0.0).
 //   * y_s_t [Mg, K]: token group i, channel k at i * K + k.
 // Pins (tests/test_oracle_formats.py): oracle_e4m3_rne against torch's
 // float8_e4m3fn conversion inside the finite range and against brute force
@@ -273,19 +275,20 @@ void oracle_quant_group_fmt(const uint16_t* v, int64_t n, int64_t stride, uint8_
   }
   if (scales) *static_cast<uint8_t*>(scale) = oracle_e8m0_ceil(static_cast<float>(s));
   else *static_cast<float*>(scale) = static_cast<float>(s);
+  // Every group, the all-zero one included (scale 1), codes v / scale: a
+  // -0.0 element therefore gets the E4M3 negative zero, as a cast of the
+  // quotient would give.
   for (int64_t i = 0; i < n; ++i) {
-    uint8_t c = 0;
-    if (amax != 0.0f) {
-      // the quotient rounded once to fp32 (exact for a power-of-two scale)
-      const float t = static_cast<float>(static_cast<double>(bf16_to_float(v[i * stride])) / s);
-      if (codes) {
-        c = oracle_e4m3_rne(t);
-      } else {
-        float r = std::nearbyint(t);
-        if (r > 127.0f) r = 127.0f;
-        if (r < -127.0f) r = -127.0f;
-        c = static_cast<uint8_t>(static_cast<int8_t>(r));
-      }
+    // the quotient rounded once to fp32 (exact for a power-of-two scale)
+    const float t = static_cast<float>(static_cast<double>(bf16_to_float(v[i * stride])) / s);
+    uint8_t c;
+    if (codes) {
+      c = oracle_e4m3_rne(t);
+    } else {
+      float r = std::nearbyint(t);
+      if (r > 127.0f) r = 127.0f;
+      if (r < -127.0f) r = -127.0f;
+      c = static_cast<uint8_t>(static_cast<int8_t>(r));
     }
     q[i * qstride] = c;
   }

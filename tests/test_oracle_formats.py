@@ -104,15 +104,19 @@ def _expected_group(bits, codes, scales):
     vals = [bf16_value(int(b)) for b in bits]
     amax = max(abs(v) for v in vals)
     if amax == 0:
-        return [0] * len(vals), (127 if scales else 1.0)
-    s = f32_round(amax / QMAX[codes])
-    if scales:
-        k = min(127, max(-127, pow2_ceil_exponent(s)))
-        s = Fraction(2) ** k
+        s, k = Fraction(1), 0
+    else:
+        s = f32_round(amax / QMAX[codes])
+        if scales:
+            k = min(127, max(-127, pow2_ceil_exponent(s)))
+            s = Fraction(2) ** k
     out = []
-    for v in vals:
+    for b, v in zip(bits, vals):
         t = f32_round(v / s)
-        out.append(e4m3_nearest(t) if codes else round_half_even(t) & 0xFF)
+        if codes:   # a quotient that is zero keeps v's sign (rationals have no -0)
+            out.append((0x80 if int(b) & 0x8000 else 0) if t == 0 else e4m3_nearest(t))
+        else:
+            out.append(round_half_even(t) & 0xFF)
     return out, ((k + 127) if scales else float(s))
 
 
@@ -123,7 +127,14 @@ def _groups(rng):
         gs.append(v)
     gs.append(np.zeros(128))
     gs.append(np.full(128, -0.75))
-    return [f64_to_bf16_bits(_bf16_exact(v)) for v in gs]
+    out = [f64_to_bf16_bits(_bf16_exact(v)) for v in gs]
+    signed_zero = np.zeros(128, np.uint16)
+    signed_zero[::3] = 0x8000             # an all-zero group with -0.0 elements
+    out.append(signed_zero)
+    mixed = out[0].copy()
+    mixed[7] = 0x8000                     # a -0.0 element in a non-zero group
+    out.append(mixed)
+    return out
 
 
 def _bf16_exact(v):
