@@ -63,7 +63,8 @@ typedef enum sdq_status {
   SDQ_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed (see sdq_last_cuda_error) */
   SDQ_ERR_TIMEOUT = 6,   /* a device-side wait hit its time limit (sdq_device_status) */
   SDQ_ERR_WORKSPACE = 7, /* the workspace given to sdq_fuse_host is too small        */
-  SDQ_ERR_TOO_LARGE = 8  /* sdq_fuse_host_noalloc: K too large for its fixed scratch  */
+  SDQ_ERR_TOO_LARGE = 8, /* sdq_fuse_host_noalloc: K too large for its fixed scratch  */
+  SDQ_ERR_FORMAT = 9     /* sdq_fuse_format: unknown bits in `format`                */
 } sdq_status;
 
 /* Largest accepted sizes: M < 2^31 (tensor-map coordinates are 32-bit) and
@@ -98,6 +99,49 @@ int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q,
 int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
                  const float* grad_input_s, const int8_t* y_q_t,
                  const float* y_s_t, int64_t M, int64_t K, int32_t group_size);
+
+/*
+ * Output formats of sdq_fuse_format, OR-ed together (0 = the page's: INT8
+ * codes, fp32 scales, y_s_t [K, ceil(M/128)]).  The page says only that the
+ * outputs feed quantized GEMMs; these variants give the layouts such GEMMs
+ * take, each following a public definition:
+ *   SDQ_FMT_E4M3     codes are OCP FP8 E4M3 bytes (sign, 4 exponent bits with
+ *                    bias 7, 3 mantissa bits, no infinities, largest finite
+ *                    448) in place of INT8: scale = fl32(amax / 448), code =
+ *                    E4M3 round-to-nearest-even of v * (1/scale), saturated
+ *                    to +-448.  Same shapes; one byte per code.
+ *   SDQ_FMT_E8M0     scales are OCP Microscaling E8M0 bytes (value 2^(e-127))
+ *                    in place of fp32: the smallest power of two not below
+ *                    fl32(amax / Qmax) (Qmax = 127 for INT8, 448 for E4M3),
+ *                    clamped to [2^-127, 2^127]; an all-zero group gets 2^0
+ *                    (byte 127).  The scale arrays hold one byte per scale
+ *                    (any alignment); every element stays inside the code
+ *                    range, and the codes are v * 2^-e exactly rounded.
+ *   SDQ_FMT_YS_MG_K  y_s_t is [ceil(M/128), K] (y_s_t[i, k] = scale of tokens
+ *                    128i.. of channel k) instead of [K, ceil(M/128)].
+ * In every format an all-zero group has scale 1 and the code of v / 1 (an
+ * E4M3 -0.0 element keeps its sign: 0x80).
+ */
+#define SDQ_FMT_E4M3 1u
+#define SDQ_FMT_E8M0 2u
+#define SDQ_FMT_YS_MG_K 4u
+
+/*
+ * sdq_fuse_format -- sdq_fuse with a chosen output format.  The code arrays
+ * are bytes (int8 or E4M3 bits); the scale arrays are fp32 (4-byte aligned)
+ * or E8M0 bytes; all other arguments, the alignment of x, grad_y and the
+ * code arrays, and the errors are those of sdq_fuse.  SDQ_ERR_FORMAT for
+ * unknown bits.  format = 0 is exactly sdq_fuse.
+ */
+int sdq_fuse_format(const void* x, const void* grad_y, void* grad_input_q,
+                    void* grad_input_s, void* y_q_t, void* y_s_t, int64_t M,
+                    int64_t K, int32_t group_size, uint32_t format, void* stream);
+
+/* The argument checks of sdq_fuse_format alone: no CUDA call, no launch. */
+int sdq_validate_format(const void* x, const void* grad_y, const void* grad_input_q,
+                        const void* grad_input_s, const void* y_q_t,
+                        const void* y_s_t, int64_t M, int64_t K,
+                        int32_t group_size, uint32_t format);
 
 /*
  * sdq_fuse_host -- the op on HOST buffers (same shapes and layouts as

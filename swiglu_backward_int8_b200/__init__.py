@@ -9,6 +9,11 @@ takes CUDA tensors x = [gate | up] (bf16 [M, 2K]) and grad_y (bf16 [M, K]) and
 writes, in place, grad_input_q (int8 [M, 2K]), grad_input_s (fp32 [M, 2K/128]),
 y_q_t (int8 [K, M]) and y_s_t (fp32 [K, ceil(M/128)]).  PyTorch supplies only
 the device memory and the current stream; the work runs in libsdq.so.
+
+Other output formats (include/sdq.h, SDQ_FMT_*) follow from the output
+tensors' dtypes: float8_e4m3fn codes (OCP FP8 E4M3), uint8 or float8_e8m0fnu
+scales (E8M0 powers of two); ``y_scale_layout="mg_k"`` gives y_s_t as
+[ceil(M/128), K].
 """
 from __future__ import annotations
 
@@ -16,13 +21,15 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import (LIB_PATH, SdqError, Status, last_cuda_error, sdq_device_status, sdq_fuse,
-                   sdq_fuse_host, sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes,
-                   sdq_validate, status_string, version)
+from ._lib import (FMT_E4M3, FMT_E8M0, FMT_YS_MG_K, LIB_PATH, SdqError, Status, last_cuda_error,
+                   sdq_device_status, sdq_fuse, sdq_fuse_format, sdq_fuse_host,
+                   sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_validate,
+                   sdq_validate_format, status_string, version)
 
 __all__ = [
     "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs",
-    "output_shapes", "sdq_fuse", "sdq_fuse_host", "sdq_fuse_host_noalloc",
+    "output_shapes", "output_format", "sdq_fuse", "sdq_fuse_format", "sdq_validate_format",
+    "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
     "sdq_fuse_host_workspace_bytes", "sdq_validate",
     "sdq_device_status", "SdqError", "Status", "status_string", "last_cuda_error", "version",
     "LIB_PATH", "GROUP_SIZE",
@@ -31,22 +38,53 @@ __all__ = [
 GROUP_SIZE = 128
 
 
-def output_shapes(M: int, K: int, group_size: int = GROUP_SIZE):
+_E8M0_DTYPES = tuple(d for d in (torch.uint8, getattr(torch, "float8_e8m0fnu", None)) if d is not None)
+_CODE_DTYPES = {"int8": (torch.int8,), "e4m3": (torch.float8_e4m3fn, torch.uint8)}
+_SCALE_DTYPES = {"fp32": (torch.float32,), "e8m0": _E8M0_DTYPES}
+_LAYOUTS = ("k_mg", "mg_k")
+
+
+def output_format(codes: str = "int8", scales: str = "fp32", y_scale_layout: str = "k_mg") -> int:
+    """FMT_* bits for the named output format."""
+    if codes not in _CODE_DTYPES or scales not in _SCALE_DTYPES or y_scale_layout not in _LAYOUTS:
+        raise ValueError(f"unknown format codes={codes!r} scales={scales!r} "
+                         f"y_scale_layout={y_scale_layout!r}")
+    return ((FMT_E4M3 if codes == "e4m3" else 0) | (FMT_E8M0 if scales == "e8m0" else 0) |
+            (FMT_YS_MG_K if y_scale_layout == "mg_k" else 0))
+
+
+def output_shapes(M: int, K: int, group_size: int = GROUP_SIZE, y_scale_layout: str = "k_mg"):
     """Shapes of (grad_input_q, grad_input_s, y_q_t, y_s_t)."""
     G = group_size
-    return (M, 2 * K), (M, 2 * (K // G)), (K, M), (K, (M + G - 1) // G)
+    Mg = (M + G - 1) // G
+    return (M, 2 * K), (M, 2 * (K // G)), (K, M), ((Mg, K) if y_scale_layout == "mg_k" else (K, Mg))
 
 
-def allocate_outputs(M: int, K: int, device, group_size: int = GROUP_SIZE):
+def allocate_outputs(M: int, K: int, device, group_size: int = GROUP_SIZE, codes: str = "int8",
+                     scales: str = "fp32", y_scale_layout: str = "k_mg"):
     """Uninitialised output tensors for one call (the op writes every element)."""
-    s = output_shapes(M, K, group_size)
-    return (torch.empty(s[0], dtype=torch.int8, device=device),
-            torch.empty(s[1], dtype=torch.float32, device=device),
-            torch.empty(s[2], dtype=torch.int8, device=device),
-            torch.empty(s[3], dtype=torch.float32, device=device))
+    output_format(codes, scales, y_scale_layout)
+    s = output_shapes(M, K, group_size, y_scale_layout)
+    cdt, sdt = _CODE_DTYPES[codes][0], _SCALE_DTYPES[scales][0]
+    return (torch.empty(s[0], dtype=cdt, device=device),
+            torch.empty(s[1], dtype=sdt, device=device),
+            torch.empty(s[2], dtype=cdt, device=device),
+            torch.empty(s[3], dtype=sdt, device=device))
 
 
-def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool):
+def _infer(kind: str, given: Optional[str], t: torch.Tensor, table) -> str:
+    if given is None:
+        for name, dts in table.items():
+            if t.dtype in dts:
+                return name
+        raise ValueError(f"cannot tell the {kind} format from dtype {t.dtype}; pass {kind}=...")
+    if given not in table:
+        raise ValueError(f"unknown {kind} format {given!r}")
+    return given
+
+
+def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", scales="fp32",
+                   y_scale_layout="k_mg"):
     if x.dim() != 2 or grad_y.dim() != 2:
         raise ValueError("x and grad_y must be 2-D")
     M, K2 = x.shape
@@ -60,10 +98,11 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool):
     if group_size != GROUP_SIZE or K % group_size:
         raise ValueError(f"group_size must be 128 and K={K} a multiple of it")
     names = ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")
-    dtypes = (torch.int8, torch.float32, torch.int8, torch.float32)
-    for name, t, shape, dt in zip(names, outs, output_shapes(M, K, group_size), dtypes):
-        if tuple(t.shape) != shape or t.dtype != dt:
-            raise ValueError(f"{name}: expected {dt} {shape}, got {t.dtype} {tuple(t.shape)}")
+    dtypes = (_CODE_DTYPES[codes], _SCALE_DTYPES[scales]) * 2
+    for name, t, shape, dts in zip(names, outs, output_shapes(M, K, group_size, y_scale_layout), dtypes):
+        if tuple(t.shape) != shape or t.dtype not in dts:
+            raise ValueError(f"{name}: expected {' or '.join(map(str, dts))} {shape}, "
+                             f"got {t.dtype} {tuple(t.shape)}")
     for name, t in zip(("x", "grad_y") + names, (x, grad_y) + tuple(outs)):
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
@@ -76,16 +115,25 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool):
 
 def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_input_q: torch.Tensor,
                                 grad_input_s: torch.Tensor, y_q_t: torch.Tensor,
-                                y_s_t: torch.Tensor, group_size: int = GROUP_SIZE) -> None:
-    """Fused SwiGLU backward + dual-axis INT8 quantization, in place, on the
-    current CUDA stream of x's device.  Raises ValueError on bad arguments and
-    SdqError on a library status."""
+                                y_s_t: torch.Tensor, group_size: int = GROUP_SIZE, *,
+                                codes: Optional[str] = None, scales: Optional[str] = None,
+                                y_scale_layout: str = "k_mg") -> None:
+    """Fused SwiGLU backward + dual-axis quantization, in place, on the
+    current CUDA stream of x's device.  The code format ("int8" or "e4m3")
+    and the scale format ("fp32" or "e8m0") follow the dtypes of
+    grad_input_q and grad_input_s unless given; ``y_scale_layout`` is "k_mg"
+    (y_s_t [K, ceil(M/128)]) or "mg_k".  Raises ValueError on bad arguments
+    and SdqError on a library status."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
-    M, K = _check_tensors(x, grad_y, outs, group_size, want_cuda=True)
+    codes = _infer("codes", codes, grad_input_q, _CODE_DTYPES)
+    scales = _infer("scales", scales, grad_input_s, _SCALE_DTYPES)
+    fmt = output_format(codes, scales, y_scale_layout)
+    M, K = _check_tensors(x, grad_y, outs, group_size, True, codes, scales, y_scale_layout)
     with torch.cuda.device(x.device):
         stream = torch.cuda.current_stream(x.device).cuda_stream
-        sdq_fuse(x.data_ptr(), grad_y.data_ptr(), grad_input_q.data_ptr(), grad_input_s.data_ptr(),
-                 y_q_t.data_ptr(), y_s_t.data_ptr(), M, K, group_size, stream)
+        sdq_fuse_format(x.data_ptr(), grad_y.data_ptr(), grad_input_q.data_ptr(),
+                        grad_input_s.data_ptr(), y_q_t.data_ptr(), y_s_t.data_ptr(), M, K,
+                        group_size, fmt, stream)
 
 
 def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
@@ -112,10 +160,12 @@ def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
             torch.cuda.current_stream(dev).synchronize()
 
 
-def run(x: torch.Tensor, grad_y: torch.Tensor, group_size: int = GROUP_SIZE
+def run(x: torch.Tensor, grad_y: torch.Tensor, group_size: int = GROUP_SIZE, codes: str = "int8",
+        scales: str = "fp32", y_scale_layout: str = "k_mg"
         ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
     """Allocate the outputs and run the op; returns (grad_input_q, grad_input_s, y_q_t, y_s_t)."""
     M, K2 = x.shape
-    outs = allocate_outputs(M, K2 // 2, x.device, group_size)
-    silu_dot_fwd_bwd_quant_fuse(x, grad_y, *outs, group_size=group_size)
+    outs = allocate_outputs(M, K2 // 2, x.device, group_size, codes, scales, y_scale_layout)
+    silu_dot_fwd_bwd_quant_fuse(x, grad_y, *outs, group_size=group_size, codes=codes,
+                                scales=scales, y_scale_layout=y_scale_layout)
     return outs

@@ -28,6 +28,10 @@ _lib.sdq_fuse.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P]
 _lib.sdq_fuse.restype = ctypes.c_int
 _lib.sdq_validate.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32]
 _lib.sdq_validate.restype = ctypes.c_int
+_lib.sdq_fuse_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctypes.c_uint32, _P]
+_lib.sdq_fuse_format.restype = ctypes.c_int
+_lib.sdq_validate_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctypes.c_uint32]
+_lib.sdq_validate_format.restype = ctypes.c_int
 _lib.sdq_fuse_host.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P, ctypes.c_size_t, _I64, _P]
 _lib.sdq_fuse_host.restype = ctypes.c_int
 _lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
@@ -56,6 +60,14 @@ class Status(enum.IntEnum):
     ERR_TIMEOUT = 6
     ERR_WORKSPACE = 7
     ERR_TOO_LARGE = 8
+    ERR_FORMAT = 9
+
+
+# Output-format bits of sdq_fuse_format (include/sdq.h): 0 = INT8 codes, fp32
+# scales, y_s_t [K, ceil(M/128)].
+FMT_E4M3 = 1       # codes are OCP FP8 E4M3 bytes
+FMT_E8M0 = 2       # scales are E8M0 bytes (powers of two)
+FMT_YS_MG_K = 4    # y_s_t is [ceil(M/128), K]
 
 
 class SdqError(RuntimeError):
@@ -91,6 +103,21 @@ def sdq_fuse(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: i
     """Raw-pointer form of the device entry point (device addresses as ints)."""
     _check(_lib.sdq_fuse(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                          group_size, stream or 0), "sdq_fuse")
+
+
+def sdq_fuse_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                    y_s_t: int, M: int, K: int, group_size: int = 128, format: int = 0,
+                    stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the device entry point with an output format (FMT_* bits)."""
+    _check(_lib.sdq_fuse_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                group_size, format, stream or 0), "sdq_fuse_format")
+
+
+def sdq_validate_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,
+                        y_s_t: int, M: int, K: int, group_size: int = 128, format: int = 0) -> int:
+    """Argument checks of sdq_fuse_format only (no CUDA call); returns the status code."""
+    return int(_lib.sdq_validate_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                        group_size, format))
 
 
 def sdq_validate(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,

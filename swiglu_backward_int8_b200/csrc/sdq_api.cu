@@ -23,6 +23,18 @@ namespace {
 constexpr int kStages = SDQ_STAGES;
 
 constexpr int kMaxDevices = 64;
+
+// One kernel per output format (SDQ_FMT_* bits 0..2).
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const sdq::Params);
+constexpr int kFormats = 8;
+KernelFn kernel_for(uint32_t format) {
+  static constexpr KernelFn table[kFormats] = {
+      sdq::fuse_kernel<kStages, false, false, false>, sdq::fuse_kernel<kStages, true, false, false>,
+      sdq::fuse_kernel<kStages, false, true, false>,  sdq::fuse_kernel<kStages, true, true, false>,
+      sdq::fuse_kernel<kStages, false, false, true>,  sdq::fuse_kernel<kStages, true, false, true>,
+      sdq::fuse_kernel<kStages, false, true, true>,   sdq::fuse_kernel<kStages, true, true, true>};
+  return table[format & (kFormats - 1)];
+}
 thread_local int t_last_cuda_error = 0;
 
 int cuda_fail(cudaError_t e) {
@@ -74,15 +86,17 @@ int current_device(DeviceState** out) {
   DeviceState& d = g_dev[dev];
   std::call_once(d.init, [&d, dev] {
     d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (d.init_err == cudaSuccess)
-      d.init_err = cudaFuncSetAttribute(sdq::fuse_kernel<kStages>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(sdq::smem_bytes<kStages>()));
-    int blocks = 0;
-    if (d.init_err == cudaSuccess)
-      d.init_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &blocks, sdq::fuse_kernel<kStages>, sdq::kThreads, sdq::smem_bytes<kStages>());
-    if (d.init_err == cudaSuccess && blocks < 1) d.init_err = cudaErrorLaunchOutOfResources;
+    for (int f = 0; f < kFormats; ++f) {
+      const auto kernel = kernel_for(static_cast<uint32_t>(f));
+      if (d.init_err == cudaSuccess)
+        d.init_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(sdq::smem_bytes<kStages>()));
+      int blocks = 0;
+      if (d.init_err == cudaSuccess)
+        d.init_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel, sdq::kThreads,
+                                                                   sdq::smem_bytes<kStages>());
+      if (d.init_err == cudaSuccess && blocks < 1) d.init_err = cudaErrorLaunchOutOfResources;
+    }
   });
   if (d.init_err != cudaSuccess) return cuda_fail(d.init_err);
   *out = &d;
@@ -104,10 +118,11 @@ int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
   return SDQ_OK;
 }
 
-// Launch on validated arguments (M > 0).  `limit_ns` = 0: the default wait
-// limit; `withhold` = 1 only for the failure-path test hook.
-int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, float* yst,
-           int64_t M, int64_t K, cudaStream_t stream, uint64_t limit_ns = 0, int withhold = 0) {
+// Launch on validated arguments (M > 0).  `format`: SDQ_FMT_* bits;
+// `limit_ns` = 0: the default wait limit; `withhold` = 1 only for the
+// failure-path test hook.
+int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void* yst, int64_t M,
+           int64_t K, uint32_t format, cudaStream_t stream, uint64_t limit_ns = 0, int withhold = 0) {
   DeviceState* d = nullptr;
   int st = current_device(&d);
   if (st != SDQ_OK) return st;
@@ -115,9 +130,9 @@ int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, 
   if ((st = make_map(&mx, x, 2 * K, M, 4 * K)) != SDQ_OK) return st;
   if ((st = make_map(&mg, gy, K, M, 2 * K)) != SDQ_OK) return st;
   sdq::Params p;
-  p.giq = giq;
+  p.giq = static_cast<int8_t*>(giq);
   p.gis = gis;
-  p.yqt = yqt;
+  p.yqt = static_cast<int8_t*>(yqt);
   p.yst = yst;
   p.M = M;
   p.K = static_cast<int32_t>(K);
@@ -141,7 +156,7 @@ int launch(const void* x, const void* gy, int8_t* giq, float* gis, int8_t* yqt, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, sdq::fuse_kernel<kStages>, mx, mg, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(format), mx, mg, p);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -196,13 +211,16 @@ const char* sdq_status_string(int status) {
     case SDQ_ERR_TIMEOUT: return "SDQ_ERR_TIMEOUT: a device-side wait ran past its limit";
     case SDQ_ERR_WORKSPACE: return "SDQ_ERR_WORKSPACE: workspace too small or misaligned";
     case SDQ_ERR_TOO_LARGE: return "SDQ_ERR_TOO_LARGE: K exceeds what fits in the fixed scratch of sdq_fuse_host_noalloc (SDQ_NOALLOC_MAX_K)";
+    case SDQ_ERR_FORMAT: return "SDQ_ERR_FORMAT: unknown bits in the output format";
     default: return "SDQ_ERR_UNKNOWN";
   }
 }
 
-int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
-                 const float* grad_input_s, const int8_t* y_q_t, const float* y_s_t, int64_t M,
-                 int64_t K, int32_t group_size) {
+int sdq_validate_format(const void* x, const void* grad_y, const void* grad_input_q,
+                        const void* grad_input_s, const void* y_q_t, const void* y_s_t, int64_t M,
+                        int64_t K, int32_t group_size, uint32_t format) {
+  if (format & ~static_cast<uint32_t>(SDQ_FMT_E4M3 | SDQ_FMT_E8M0 | SDQ_FMT_YS_MG_K))
+    return SDQ_ERR_FORMAT;
   if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
   if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
     return SDQ_ERR_SHAPE;
@@ -213,16 +231,30 @@ int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
   const uintptr_t a16 = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(grad_y) |
                         reinterpret_cast<uintptr_t>(grad_input_q) | reinterpret_cast<uintptr_t>(y_q_t);
   const uintptr_t a4 = reinterpret_cast<uintptr_t>(grad_input_s) | reinterpret_cast<uintptr_t>(y_s_t);
-  if ((a16 & 15u) || (a4 & 3u)) return SDQ_ERR_ALIGN;
+  if ((a16 & 15u) || (!(format & SDQ_FMT_E8M0) && (a4 & 3u))) return SDQ_ERR_ALIGN;
   return SDQ_OK;
+}
+
+int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
+                 const float* grad_input_s, const int8_t* y_q_t, const float* y_s_t, int64_t M,
+                 int64_t K, int32_t group_size) {
+  return sdq_validate_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, 0);
+}
+
+int sdq_fuse_format(const void* x, const void* grad_y, void* grad_input_q, void* grad_input_s,
+                    void* y_q_t, void* y_s_t, int64_t M, int64_t K, int32_t group_size,
+                    uint32_t format, void* stream) {
+  const int st = sdq_validate_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+                                     group_size, format);
+  if (st != SDQ_OK || M == 0) return st;
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, format,
+                static_cast<cudaStream_t>(stream));
 }
 
 int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q, float* grad_input_s,
              int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K, int32_t group_size, void* stream) {
-  const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
-  if (st != SDQ_OK || M == 0) return st;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
-                static_cast<cudaStream_t>(stream));
+  return sdq_fuse_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, 0,
+                         stream);
 }
 
 size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows) {
@@ -293,9 +325,8 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
     SDQ_CHECK(cudaEventRecord(d->in_ready[b], d->h2d));
     // kernel on the caller's stream
     SDQ_CHECK(cudaStreamWaitEvent(cs, d->in_ready[b], 0));
-    st = launch(base + L.x, base + L.gy, reinterpret_cast<int8_t*>(base + L.giq),
-                reinterpret_cast<float*>(base + L.gis), reinterpret_cast<int8_t*>(base + L.yqt),
-                reinterpret_cast<float*>(base + L.yst), mc, K, cs);
+    st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt, base + L.yst, mc,
+                K, 0, cs);
     if (st != SDQ_OK) return st;
     SDQ_CHECK(cudaEventRecord(d->out_ready[b], cs));
     // device -> host
@@ -386,10 +417,8 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
     if ((e = cudaMemcpyAsync(base + L.gy, gh + m0 * 2 * K, size_t(mc) * 2 * K,
                              cudaMemcpyHostToDevice, cs)) != cudaSuccess)
       return cuda_fail(e);
-    const int st = launch(base + L.x, base + L.gy, reinterpret_cast<int8_t*>(base + L.giq),
-                          reinterpret_cast<float*>(base + L.gis),
-                          reinterpret_cast<int8_t*>(base + L.yqt),
-                          reinterpret_cast<float*>(base + L.yst), mc, K, cs);
+    const int st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt,
+                          base + L.yst, mc, K, 0, cs);
     if (st != SDQ_OK) return st;
     if ((e = cudaMemcpyAsync(grad_input_q + m0 * 2 * K, base + L.giq, size_t(mc) * 2 * K,
                              cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
@@ -414,7 +443,7 @@ int sdq_fuse_test_stall(const void* x, const void* grad_y, int8_t* grad_input_q,
   const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
   if (st != SDQ_OK || M == 0) return st;
   if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000) return SDQ_ERR_SHAPE;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, 0,
                 static_cast<cudaStream_t>(stream), static_cast<uint64_t>(wait_limit_ns), 1);
 }
 

@@ -72,11 +72,16 @@ constexpr int kDevTimeout = 1;  // bit in the device status word
 // Device status word: OR of kDev* bits; read and cleared by sdq_device_status().
 __device__ int g_sdq_dev_status;
 
+// Output formats, template parameters of the kernel (so the page's format
+// runs the same instructions as a kernel built for it alone): codes INT8
+// (the page's) or OCP FP8 E4M3; scales fp32 (the page's) or E8M0 bytes (the
+// smallest power of two not below amax/Qmax); y_s_t [K, Mg] (the page's) or
+// [Mg, K].
 struct Params {
-  int8_t* giq;   // [M, 2K]
-  float* gis;    // [M, 2K/128]
-  int8_t* yqt;   // [K, M]
-  float* yst;    // [K, Mg]
+  int8_t* giq;   // [M, 2K] code bytes
+  void* gis;     // [M, 2K/128] fp32 or E8M0 bytes
+  int8_t* yqt;   // [K, M] code bytes
+  void* yst;     // [K, Mg] or [Mg, K], fp32 or E8M0 bytes
   int64_t M;
   int32_t K;
   int32_t Kg;
@@ -91,7 +96,7 @@ template <int STAGES>
 struct Smem {
   alignas(128) uint8_t ring[STAGES][kStageBytes];  // [gate | up | grad_y], each [64][128] bf16
   alignas(16) uint8_t ytile[kYBuf][kYBytes];       // bf16 y [token][channel], chunks swizzled
-  alignas(16) float2 scale_tab[128];               // (fl((1+m/128)/127), 1/that) per bf16 mantissa m
+  alignas(16) float2 scale_tab[128];               // per bf16 mantissa m: scale and inverse for 2^0 (see group_scale)
   alignas(8) uint64_t full[STAGES];
   alignas(8) uint64_t y_ready[kYBuf];              // all threads wrote their rows of the y tile
   alignas(8) uint64_t y_free[kYBuf];               // all threads finished reading the y tile
@@ -169,83 +174,133 @@ __device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t d
 }
 
 // Scale and inverse scale of a group from its amax, given as non-negative
-// bf16 bits: scale = amax/127 correctly rounded, inv = 1/scale correctly
-// rounded; an all-zero group gets scale 1.  A bf16 amax is (1 + m/128) * 2^e,
-// so scale = fl((1 + m/128)/127) * 2^e exactly whenever that is a normal
-// float: the table holds the two mantissa-dependent quotients and the power of
-// two goes into the exponent field.
-// Tiny groups (amax < 2^-119, bf16 exponent field < 8) take the quotients
-// directly; their 1/scale can exceed the float range, so for them the
-// returned inverse is meant for values pre-multiplied by kTinyPre (= 2^64) and
-// comes back negated as a marker: (v * 2^64) * fl(1/(scale * 2^64)) is the
-// same real number as v * fl(1/scale).
+// bf16 bits, for codes up to Qmax (127 for INT8, 448 for E4M3):
+//   fp32 scales: scale = fl(amax / Qmax), inv = fl(1 / scale);
+//   E8M0 scales: scale = the smallest power of two >= fl(amax / Qmax),
+//                clamped to [2^-127, 2^127], inv = 1 / scale (exact);
+// an all-zero group gets scale 1.  A bf16 amax is (1 + m/128) * 2^e, and
+// fl(amax / Qmax) = fl((1 + m/128) / Qmax) * 2^e exactly whenever both are
+// normal floats; so a 128-entry table holds, per mantissa m, the scale and
+// inverse for e = 0 (fl((1 + m/128)/Qmax) and its reciprocal, or the power of
+// two above it and its reciprocal), and 2^e goes into the exponent fields.
+// That holds for every bf16 exponent field >= kTableEx; smaller amaxes (below
+// 2^-117) take the out-of-line IEEE path.  There, with fp32 scales, 1/scale can
+// exceed the float range, so the returned inverse is meant for values
+// pre-multiplied by kTinyPre (= 2^64) and comes back negated as a marker:
+// (v * 2^64) * fl(1/(scale * 2^64)) is the same real number as v * fl(1/scale).
+// E8M0 inverses are at most 2^127 and need no marker.
 constexpr float kTinyPre = 18446744073709551616.0f;  // 2^64
+constexpr uint32_t kTableEx = 10;
 
-// The rare branch, kept out of line so the common path stays short.
-__device__ __noinline__ float2 tiny_group_scale(uint32_t abits) {
-  if (abits == 0u) return make_float2(1.0f, 1.0f);
-  const float scale = __fdiv_rn(__uint_as_float(abits << 16), 127.0f);
-  return make_float2(scale, -__frcp_rn(scale * kTinyPre));
+template <bool kE4M3>
+__host__ __device__ constexpr float qmax() { return kE4M3 ? 448.0f : 127.0f; }
+
+// Exponent k of the smallest power of two >= s (s > 0, finite, subnormals included).
+__device__ __forceinline__ int ceil_log2(float s) {
+  const uint32_t b = __float_as_uint(s);
+  if (b >= 0x00800000u) return static_cast<int>(b >> 23) - 127 + ((b & 0x007FFFFFu) != 0u ? 1 : 0);
+  return (31 - __clz(static_cast<int>(b))) - 149 + ((b & (b - 1u)) != 0u ? 1 : 0);
 }
 
+// 2^k as a float for -127 <= k <= 127 (2^-127 is subnormal).
+__device__ __forceinline__ float pow2f(int k) {
+  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Table entry for mantissa m (scale and inverse for a bf16 exponent field of 127).
+template <bool kE4M3, bool kE8M0>
+__device__ __forceinline__ float2 scale_table_entry(int m) {
+  const float t = __fdiv_rn(1.0f + static_cast<float>(m) * (1.0f / 128.0f), qmax<kE4M3>());
+  if (!kE8M0) return make_float2(t, __frcp_rn(t));
+  const int k = ceil_log2(t);
+  return make_float2(pow2f(k), pow2f(-k));
+}
+
+// The rare branch, kept out of line so the common path stays short.
+template <bool kE4M3, bool kE8M0>
+__device__ __noinline__ float2 tiny_group_scale(uint32_t abits) {
+  if (abits == 0u) return make_float2(1.0f, 1.0f);
+  const float s = __fdiv_rn(__uint_as_float(abits << 16), qmax<kE4M3>());
+  if (!kE8M0) return make_float2(s, -__frcp_rn(s * kTinyPre));
+  const int k = max(ceil_log2(s), -127);   // a bf16 amax never needs more than 2^122
+  return make_float2(pow2f(k), pow2f(-k));
+}
+
+template <bool kE4M3, bool kE8M0>
 __device__ __forceinline__ void group_scale(uint32_t abits, const float2* tab, float& scale,
                                             float& inv_marked) {
   const uint32_t ex = abits >> 7;
-  if (ex >= 8u) {
+  if (ex >= kTableEx) {
     const float2 t = tab[abits & 127u];
     const int sh = (static_cast<int>(ex) - 127) << 23;
     scale = __int_as_float(__float_as_int(t.x) + sh);
     inv_marked = __int_as_float(__float_as_int(t.y) - sh);
   } else {
-    const float2 r = tiny_group_scale(abits);
+    const float2 r = tiny_group_scale<kE4M3, kE8M0>(abits);
     scale = r.x;
     inv_marked = r.y;
   }
 }
 
-// Round-half-even codes of a bf16 pair times `inv` (each half pre-multiplied
-// by `pre` first); each code is the low byte of its float's bits.
-template <bool kTiny>
+// A scale into an fp32 array, or as its E8M0 byte (a power of two in
+// [2^-127, 2^127] carries its byte in the float's exponent field; 2^-127,
+// subnormal, gives 0).
+template <bool kE8M0>
+__device__ __forceinline__ void store_scale(void* base, int64_t idx, float scale) {
+  if (kE8M0) static_cast<uint8_t*>(base)[idx] = static_cast<uint8_t>(__float_as_uint(scale) >> 23);
+  else static_cast<float*>(base)[idx] = scale;
+}
+
+// A bf16 pair times `inv` (each half pre-multiplied by `pre` first).  INT8:
+// round-half-even codes, each the low byte of its float's bits (the constant
+// 1.5 * 2^23 inside the fused multiply-add rounds to an integer).  E4M3: the
+// two fp32 products.
+template <bool kE4M3, bool kTiny>
 __device__ __forceinline__ float2 quant2(uint32_t v, float2 inv, float2 pre) {
   float2 x = unpack2(v);
   if (kTiny) x = __fmul2_rn(x, pre);
+  if (kE4M3) return __fmul2_rn(x, inv);
   return __ffma2_rn(x, inv, make_float2(12582912.0f, 12582912.0f));
 }
 
-// Sixteen int8 codes of one row piece (8 bf16 pairs) with one inverse scale.
-template <bool kTiny>
+// Four codes (in byte order a.x, a.y, b.x, b.y) from two quant2 results.
+template <bool kE4M3>
+__device__ __forceinline__ uint32_t pack_codes(float2 a, float2 b) {
+  if (kE4M3) return e4m3x4(a.x, a.y, b.x, b.y);
+  return pack_low_bytes(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
+                        __float_as_uint(b.y));
+}
+
+// Sixteen codes of one row piece (8 bf16 pairs) with one inverse scale.
+template <bool kE4M3, bool kTiny>
 __device__ __forceinline__ uint4 quant16(const uint32_t (&v)[8], float inv) {
   const float2 iv = make_float2(inv, inv);
   const float2 pre = make_float2(kTinyPre, kTinyPre);
   uint32_t w[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 a = quant2<kTiny>(v[2 * k], iv, pre);
-    const float2 b = quant2<kTiny>(v[2 * k + 1], iv, pre);
-    w[k] = pack_low_bytes(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
-                          __float_as_uint(b.y));
-  }
+  for (int k = 0; k < 4; ++k)
+    w[k] = pack_codes<kE4M3>(quant2<kE4M3, kTiny>(v[2 * k], iv, pre),
+                             quant2<kE4M3, kTiny>(v[2 * k + 1], iv, pre));
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // Column pass: 16 tokens x 2 channels (one bf16 pair per token) -> two
 // 16-byte code rows (low channel, high channel).
-template <bool kTiny>
+template <bool kE4M3, bool kTiny>
 __device__ __forceinline__ void quant_cols(const uint32_t (&v)[16], float2 inv, float2 pre,
                                            uint4& lo, uint4& hi) {
-  uint32_t bl[16], bh[16];
+  float2 q[16];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const float2 q = quant2<kTiny>(v[t], inv, pre);
-    bl[t] = __float_as_uint(q.x);
-    bh[t] = __float_as_uint(q.y);
+  for (int t = 0; t < 16; ++t) q[t] = quant2<kE4M3, kTiny>(v[t], inv, pre);
+  uint32_t wl[4], wh[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    // low channel: the .x of tokens 4w..4w+3; high channel: the .y
+    wl[w] = pack_codes<kE4M3>(make_float2(q[4 * w].x, q[4 * w + 1].x), make_float2(q[4 * w + 2].x, q[4 * w + 3].x));
+    wh[w] = pack_codes<kE4M3>(make_float2(q[4 * w].y, q[4 * w + 1].y), make_float2(q[4 * w + 2].y, q[4 * w + 3].y));
   }
-  lo = make_uint4(pack_low_bytes(bl[0], bl[1], bl[2], bl[3]), pack_low_bytes(bl[4], bl[5], bl[6], bl[7]),
-                  pack_low_bytes(bl[8], bl[9], bl[10], bl[11]),
-                  pack_low_bytes(bl[12], bl[13], bl[14], bl[15]));
-  hi = make_uint4(pack_low_bytes(bh[0], bh[1], bh[2], bh[3]), pack_low_bytes(bh[4], bh[5], bh[6], bh[7]),
-                  pack_low_bytes(bh[8], bh[9], bh[10], bh[11]),
-                  pack_low_bytes(bh[12], bh[13], bh[14], bh[15]));
+  lo = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+  hi = make_uint4(wh[0], wh[1], wh[2], wh[3]);
 }
 
 // 16 code bytes to a y_q_t row piece that may be cut short by the token count
@@ -283,6 +338,7 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uin
 // 16kc .. 16kc+15 of the bf16 y tile -> column amax over the 8 threads that
 // share the channels, the two column scales, codes, two 16-byte pieces of
 // y_q_t rows.
+template <bool kE4M3, bool kE8M0, bool kYsMgK>
 __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab, const Params& p,
                                             int i, int j, int64_t row0, int valid, int cp, int kc) {
   constexpr unsigned kFull = 0xffffffffu;
@@ -298,18 +354,19 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 4));
   m &= 0x7FFF7FFFu;
   float s_lo, i_lo, s_hi, i_hi;
-  group_scale(m & 0xFFFFu, tab, s_lo, i_lo);
-  group_scale(m >> 16, tab, s_hi, i_hi);
+  group_scale<kE4M3, kE8M0>(m & 0xFFFFu, tab, s_lo, i_lo);
+  group_scale<kE4M3, kE8M0>(m >> 16, tab, s_hi, i_hi);
   const int ch = j * kG + 2 * cp;
-  if (kc == 0) p.yst[int64_t(ch) * p.Mg + i] = s_lo;
-  if (kc == 1) p.yst[int64_t(ch + 1) * p.Mg + i] = s_hi;
+  if (kc < 2)
+    store_scale<kE8M0>(p.yst, kYsMgK ? int64_t(i) * p.K + ch + kc : int64_t(ch + kc) * p.Mg + i,
+                       kc ? s_hi : s_lo);
   uint4 lo, hi;
   if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
     // pre-multiply only the tiny channels; the others use factor 1
-    quant_cols<true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
-                     make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f), lo, hi);
+    quant_cols<kE4M3, true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
+                            make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f), lo, hi);
   } else {
-    quant_cols<false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
+    quant_cols<kE4M3, false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
   }
   const int tok = 16 * kc;
   if (tok < valid) {
@@ -320,7 +377,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   }
 }
 
-template <int STAGES>
+template <int STAGES, bool kE4M3, bool kE8M0, bool kYsMgK>
 __global__ void __launch_bounds__(kThreads, 1)
     fuse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy,
                 const Params p) {
@@ -345,10 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t total = static_cast<uint32_t>(my_tiles) * kStagesPerTile;
   const uint64_t pol = l2_policy_evict_first();  // inputs are read exactly once
 
-  if (tid < 128) {
-    const float sc = __fdiv_rn(1.0f + static_cast<float>(tid) * (1.0f / 128.0f), 127.0f);
-    s.scale_tab[tid] = make_float2(sc, __frcp_rn(sc));
-  }
+  if (tid < 128) s.scale_tab[tid] = scale_table_entry<kE4M3, kE8M0>(tid);
   if (tid == 0) {
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_gy);
@@ -399,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* yt = s.ytile[yb];
     // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
     int8_t* giq_t = p.giq + row0 * (2 * int64_t(K)) + j * kG;
-    float* gis_t = p.gis + row0 * (2 * Kg) + j;
+    const int64_t gis_t = row0 * (2 * Kg) + j;   // scale index of (row0, group j)
 
     // ================= row pass over the tile's two stages
 #pragma unroll
@@ -476,21 +530,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- the row's two scales, computed by each of its 8 lanes (no shuffles
       // on this path); lanes 0 and 1 of the row store them
       float sg, ig, su, iu;
-      group_scale(pr >> 16, tab, sg, ig);
-      group_scale(pr & 0xFFFFu, tab, su, iu);
+      group_scale<kE4M3, kE8M0>(pr >> 16, tab, sg, ig);
+      group_scale<kE4M3, kE8M0>(pr & 0xFFFFu, tab, su, iu);
       const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
-      if (cq < 2 && rbase + rr < valid) gis_t[(rbase + rr) * (2 * Kg) + cq * Kg] = cq ? su : sg;
+      if (cq < 2 && rbase + rr < valid)
+        store_scale<kE8M0>(p.gis, gis_t + (rbase + rr) * (2 * Kg) + cq * Kg, cq ? su : sg);
 
       // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
       const int r = rbase + rr;   // this lane's row within the tile
       if (r < valid) {
         uint4 og, ou;
         if (__any_sync(__activemask(), ig < 0.0f || iu < 0.0f)) {   // a tiny group in this warp (rare)
-          og = (ig < 0.0f) ? quant16<true>(dgp, -ig) : quant16<false>(dgp, ig);
-          ou = (iu < 0.0f) ? quant16<true>(dup, -iu) : quant16<false>(dup, iu);
+          og = (ig < 0.0f) ? quant16<kE4M3, true>(dgp, -ig) : quant16<kE4M3, false>(dgp, ig);
+          ou = (iu < 0.0f) ? quant16<kE4M3, true>(dup, -iu) : quant16<kE4M3, false>(dup, iu);
         } else {
-          og = quant16<false>(dgp, ig);
-          ou = quant16<false>(dup, iu);
+          og = quant16<kE4M3, false>(dgp, ig);
+          ou = quant16<kE4M3, false>(dup, iu);
         }
         int8_t* dst = giq_t + r * (2 * K);
         st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
@@ -508,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[pb]), ((k - 1) / kYBuf) & 1, lim,
                                            abort_flag));
       if (!ok) break;
-      column_pass(s.ytile[pb], tab, p, pi, pj, prow0, pvalid, cp, kc);
+      column_pass<kE4M3, kE8M0, kYsMgK>(s.ytile[pb], tab, p, pi, pj, prow0, pvalid, cp, kc);
       mbar_arrive(smem_u32(&s.y_free[pb]));
     }
     pi = i;
@@ -522,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k = my_tiles - 1;
     ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[k % kYBuf]), (k / kYBuf) & 1, lim,
                                          abort_flag));
-    if (ok) column_pass(s.ytile[k % kYBuf], tab, p, pi, pj, prow0, pvalid, cp, kc);
+    if (ok) column_pass<kE4M3, kE8M0, kYsMgK>(s.ytile[k % kYBuf], tab, p, pi, pj, prow0, pvalid, cp, kc);
   }
 
   __syncthreads();   // every thread arrives here, whether it stopped early or not

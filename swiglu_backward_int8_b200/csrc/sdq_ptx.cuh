@@ -188,6 +188,20 @@ __device__ __forceinline__ uint32_t quant_bits(float v, float inv) {
   return __float_as_uint(fmaf(v, inv, 12582912.0f));
 }
 
+// Four floats -> four OCP E4M3 codes (round to nearest even, magnitudes
+// above 448 saturated), a in byte 0.  cvt.rn.satfinite.e4m3x2.f32 puts its
+// first source in the upper byte of the pair.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n}\n"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 // Low bytes of four words -> one word (a in byte 0).
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);

@@ -120,3 +120,121 @@ def tile_of(outputs, M, K, i, j, G=128):
     tq = np.concatenate([np.asarray(q[:, c]), np.asarray(q[:, K + j * G:K + (j + 1) * G])], axis=1)
     ts = np.stack([np.asarray(gis[r0:r1, j]), np.asarray(gis[r0:r1, Kg + j])], axis=1)
     return tq, ts, np.asarray(yqt[c, r0:r1]), np.asarray(yst[c, i:i + 1])
+
+
+# ---- output formats (codes: 0 INT8, 1 E4M3; scales: 0 fp32, 1 E8M0;
+# ys_layout: 0 y_s_t [K, Mg], 1 [Mg, K]) -------------------------------------
+#
+# Tolerances for the formats, from the same arithmetic as above: a value that
+# rounds to the other bf16 neighbour, or a quotient next to a rounding
+# boundary of the code, moves a code to the adjacent one; with E8M0 scales a
+# flipped amax can also move the group's power of two by one step.  So:
+# codes equal on all but 0.1 % of the elements, and every dequantized value
+# (code x scale) within one code step (of either side) of the oracle's;
+# fp32 scales within 2^-7 relative, E8M0 bytes within 1 and equal on all but
+# 0.1 %.  E4M3 has two zero codes of one value, +0 (0x00) and -0 (0x80); where
+# sigma(g) underflows to 0 in fp32 (g < -88) but not in fp64, the kernel's
+# product is an exact zero signed by the other factors while the oracle's
+# tiny value rounds to the zero of its own sign, so the two zeros count as
+# equal (and are reported as n_signed_zero).
+
+SENTINEL_CODE = {0: 0x80, 1: 0x7F}     # INT8 -128; E4M3 NaN: neither is ever written
+SENTINEL_E8M0 = 0xFF                   # E8M0 NaN: scales stop at 2^127 (byte 254)
+
+
+def _e4m3_values():
+    from tests.exact import e4m3_table
+    v = np.full(256, np.nan)
+    for val, c in e4m3_table():
+        v[c] = float(val)
+        v[c | 0x80] = -float(val)
+    return v
+
+
+E4M3_VALUE = _e4m3_values()
+
+
+def run_cuda_fmt(x_u16: np.ndarray, gy_u16: np.ndarray, codes: int, scales: int, ys_layout: int):
+    """The device entry point in a chosen format, on guarded outputs; returns
+    numpy (code bytes, scales, code bytes, scales) like the format oracle."""
+    import swiglu_backward_int8_b200 as sdq
+    M, K = gy_u16.shape
+    x = to_device_bf16(x_u16)
+    gy = to_device_bf16(gy_u16)
+    shp = oracle.output_shapes_fmt(M, K, 128, ys_layout)
+    sq = SENTINEL_CODE[codes]
+    mk_s = (lambda s: Guarded(s, torch.uint8, SENTINEL_E8M0)) if scales else \
+        (lambda s: Guarded(s, torch.float32, float("nan")))
+    outs = [Guarded(shp[0], torch.uint8, sq), mk_s(shp[1]), Guarded(shp[2], torch.uint8, sq), mk_s(shp[3])]
+    fmt = (sdq.FMT_E4M3 if codes else 0) | (sdq.FMT_E8M0 if scales else 0) | \
+        (sdq.FMT_YS_MG_K if ys_layout else 0)
+    sdq.sdq_fuse_format(x.data_ptr(), gy.data_ptr(), *(o.t.data_ptr() for o in outs), M, K, 128, fmt,
+                        torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert sdq.sdq_device_status() == 0
+    for o, name in zip(outs, ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")):
+        assert o.guards_intact(), f"{name}: guard bytes overwritten"
+    giq, gis, yqt, yst = (o.t.cpu().numpy() for o in outs)
+    assert not (giq == sq).any() and not (yqt == sq).any(), "codes left unwritten"
+    if scales:
+        assert not (gis == SENTINEL_E8M0).any() and not (yst == SENTINEL_E8M0).any(), "scales left unwritten"
+    else:
+        assert np.isfinite(gis).all() and np.isfinite(yst).all(), "scales left unwritten"
+    return giq, gis, yqt, yst
+
+
+def _code_values(q, codes):
+    return E4M3_VALUE[q] if codes else q.view(np.int8).astype(np.float64)
+
+
+def _code_step(vals, codes):
+    if not codes:
+        return np.ones_like(vals)
+    e = np.floor(np.log2(np.maximum(np.abs(vals), 2.0 ** -6)))
+    return 2.0 ** (e - 3)       # E4M3 spacing at |v| (2^-9 below the normal range)
+
+
+def _scale_values(s, scales):
+    return np.ldexp(1.0, s.astype(np.int64) - 127) if scales else s.astype(np.float64)
+
+
+def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where=""):
+    """Assert the format tolerances; returns mismatch statistics."""
+    giq, gis, yqt, yst = got
+    rq, rs, ryq, rys = ref
+    if ys_layout:
+        yst, rys = yst.T, rys.T
+    stats = {}
+    for name, a, b in (("grad_input_s", gis, rs), ("y_s_t", yst, rys)):
+        assert a.shape == b.shape, (name, a.shape, b.shape)
+        nd = int((a != b).sum())
+        stats[name] = {"n_diff": nd}
+        if scales:
+            d = np.abs(a.astype(np.int16) - b.astype(np.int16))
+            assert d.max(initial=0) <= 1, f"{where} {name}: E8M0 bytes differ by {d.max()}"
+            assert nd <= 1e-3 * a.size, f"{where} {name}: {nd} of {a.size} E8M0 scales differ"
+        else:
+            rel = np.abs(a.astype(np.float64) - b.astype(np.float64)) / np.abs(b.astype(np.float64))
+            assert rel.max(initial=0) <= SCALE_MAX_REL, f"{where} {name}: max rel = {rel.max()}"
+    G = 128
+    M = giq.shape[0]
+    for name, a, b, sa, sb in (("grad_input_q", giq, rq, np.repeat(gis, G, axis=1), np.repeat(rs, G, axis=1)),
+                               ("y_q_t", yqt, ryq, np.repeat(yst, G, axis=1)[:, :M],
+                                np.repeat(rys, G, axis=1)[:, :M])):
+        assert a.shape == b.shape, (name, a.shape, b.shape)
+        differ = a != b
+        signed_zero = np.zeros_like(differ)
+        if codes:
+            signed_zero = differ & ((a & 0x7F) == 0) & ((b & 0x7F) == 0)
+            differ &= ~signed_zero
+        nd = int(differ.sum())
+        va, vb = _code_values(a, codes), _code_values(b, codes)
+        fa, fb = _scale_values(sa, scales), _scale_values(sb, scales)
+        tol = _code_step(va, codes) * fa + _code_step(vb, codes) * fb
+        err = np.abs(va * fa - vb * fb)
+        bad = err > tol
+        stats[name] = {"n_diff": nd, "frac_diff": nd / max(1, a.size), "n_out_of_step": int(bad.sum()),
+                       "n_signed_zero": int(signed_zero.sum())}
+        assert not bad.any(), f"{where} {name}: {int(bad.sum())} values more than a step apart"
+        assert nd <= 1e-3 * a.size, f"{where} {name}: {nd} of {a.size} codes differ"
+    return stats

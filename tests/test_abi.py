@@ -108,3 +108,49 @@ def test_torch_wrapper_argument_checks():
         sdq.silu_dot_fwd_bwd_quant_fuse(x.float(), gy, *outs)
     with pytest.raises(ValueError):
         sdq.silu_dot_fwd_bwd_quant_fuse(x, gy[:, :64], *outs)
+
+
+@pytest.mark.parametrize("fmt,args,status", [
+    (0, dict(), 0),
+    (7, dict(), 0),
+    (8, dict(), 9),                        # unknown bit
+    (1 << 31, dict(), 9),
+    (2, dict(grad_input_s=A + 1, y_s_t=A + 3), 0),   # E8M0 scales are bytes: any alignment
+    (0, dict(grad_input_s=A + 1), 4),
+    (1, dict(y_s_t=A + 2), 4),             # E4M3 codes with fp32 scales: 4-byte scales
+    (6, dict(grad_input_q=A + 1), 4),      # code arrays stay 16-byte aligned
+    (3, dict(group_size=64), 2),
+    (5, dict(M=0, x=0), 0),
+])
+def test_validate_format_statuses(fmt, args, status):
+    import swiglu_backward_int8_b200 as sdq
+    a = dict(x=A, grad_y=A, grad_input_q=A, grad_input_s=A, y_q_t=A, y_s_t=A, M=256, K=256,
+             group_size=128)
+    a.update(args)
+    assert sdq.sdq_validate_format(a["x"], a["grad_y"], a["grad_input_q"], a["grad_input_s"],
+                                   a["y_q_t"], a["y_s_t"], a["M"], a["K"], a["group_size"],
+                                   fmt) == status
+
+
+def test_format_names_shapes_and_dtypes():
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    assert sdq.output_format() == 0
+    assert sdq.output_format("e4m3", "e8m0", "mg_k") == 7
+    assert sdq.output_format(scales="e8m0") == sdq.FMT_E8M0
+    with pytest.raises(ValueError):
+        sdq.output_format("fp4")
+    q, s, yq, ys = sdq.allocate_outputs(300, 256, "cpu", codes="e4m3", scales="e8m0",
+                                        y_scale_layout="mg_k")
+    assert q.dtype == torch.float8_e4m3fn and yq.dtype == torch.float8_e4m3fn
+    assert s.dtype == torch.uint8 and ys.dtype == torch.uint8
+    assert tuple(q.shape) == (300, 512) and tuple(s.shape) == (300, 4)
+    assert tuple(yq.shape) == (256, 300) and tuple(ys.shape) == (3, 256)
+    x = torch.zeros(300, 512, dtype=torch.bfloat16)
+    gy = torch.zeros(300, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):     # host tensors: the device entry refuses before any call
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, q, s, yq, ys, y_scale_layout="mg_k")
+    with pytest.raises(ValueError):     # [K, Mg] scales where [Mg, K] was asked for
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, q, s, yq, ys.T.contiguous(), y_scale_layout="mg_k")
+    with pytest.raises(ValueError):     # E4M3 codes with INT8 asked for
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, q, s, yq, ys, codes="int8", y_scale_layout="mg_k")
