@@ -65,6 +65,13 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0 = min(steps, 50)")
+    ap.add_argument("--codes", choices=["int8", "e4m3"], default="int8",
+                    help="code format of the timed calls (the page's: int8)")
+    ap.add_argument("--scales", choices=["fp32", "e8m0"], default="fp32",
+                    help="scale format of the timed calls (the page's: fp32)")
+    ap.add_argument("--y-scale-layout", choices=["k_mg", "mg_k"], default="k_mg")
+    ap.add_argument("--all-formats", action="store_true",
+                    help="also time every output format on the workload and add a per_format list")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -258,11 +265,23 @@ def _to_device_bf16(a_u16, device):
     return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device):
+PAGE_FORMAT = ("int8", "fp32", "k_mg")
+
+
+def format_name(fmt) -> str:
+    return "-".join(fmt)
+
+
+def scale_bytes(fmt) -> int:
+    return 1 if fmt[1] == "e8m0" else 4
+
+
+def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, fmt=PAGE_FORMAT):
     import torch
     import swiglu_backward_int8_b200 as sdq
     M, K = w.M, w.K
-    footprint = w.algorithmic_bytes()
+    codes, scales, layout = fmt
+    footprint = w.algorithmic_bytes(scale_bytes(fmt))
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nsets = max(1, -(-3 * l2 // footprint))
     x0, g0 = _to_device_bf16(x_np, device), _to_device_bf16(gy_np, device)
@@ -270,12 +289,14 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device):
     for s in range(nsets):
         xs = x0 if s == 0 else x0.clone()
         gs = g0 if s == 0 else g0.clone()
-        sets.append((xs, gs, sdq.allocate_outputs(M, K, device)))
+        sets.append((xs, gs, sdq.allocate_outputs(M, K, device, codes=codes, scales=scales,
+                                                  y_scale_layout=layout)))
     stream = torch.cuda.current_stream(device)
 
     def call(k):
         xs, gs, outs = sets[k % nsets]
-        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs)
+        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, codes=codes, scales=scales,
+                                        y_scale_layout=layout)
 
     for k in range(warmup):
         call(k)
@@ -359,17 +380,20 @@ def run_sdq(args):
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     time.sleep(0.3)
-    ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device)
+    fmt = (args.codes, args.scales, args.y_scale_layout)
+    ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, fmt)
     clocks = sampler.summary(t0, t1)
     sampler.stop()
     ms_max = parallel.max_over_ranks(ms, device)
     per_step_ms = ms_max / args.steps
-    bytes_step = w.algorithmic_bytes()
+    bytes_step = w.algorithmic_bytes(scale_bytes(fmt))
     value = parallel.aggregate_gbs(bytes_step * args.steps, world, ms_max)
     achieved = bytes_step / (per_step_ms * 1e-3) / 1e9
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and fmt != PAGE_FORMAT:
+        e2e = {"unavailable": "the host-buffer entry points write the page's format only"}
+    elif not args.no_e2e:
         e2e_steps = args.e2e_steps or min(args.steps, 50)
         e = measure_e2e(wr, x_np, gy_np, e2e_steps, device)
         e_ms = parallel.max_over_ranks(e["ms_per_step"], device)
@@ -391,19 +415,36 @@ def run_sdq(args):
                         "steps": osteps, "buffer_sets": ons})
             del ox, og
 
+    per_fmt = None
+    if args.all_formats:
+        per_fmt = []
+        for c in ("int8", "e4m3"):
+            for sc in ("fp32", "e8m0"):
+                for lay in ("k_mg", "mg_k"):
+                    f = (c, sc, lay)
+                    fms, _, _ = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, f)
+                    fms = parallel.max_over_ranks(fms, device)
+                    us = fms / args.steps * 1e3
+                    fb = w.algorithmic_bytes(scale_bytes(f))
+                    gbs = fb / (us * 1e-6) / 1e9
+                    per_fmt.append({"format": format_name(f), "us_per_call": us, "GB_s": gbs,
+                                    "frac_of_measured_hbm": gbs / peak,
+                                    "algorithmic_bytes_per_launch": fb})
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0)
 
     if rank == 0:
-        traffic = recorded_traffic(w.name)
+        traffic = recorded_traffic(w.name) if fmt == PAGE_FORMAT else None
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
             "us_per_call": per_step_ms * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "K": w.K, "group_size": w.group_size,
-                       "io": "bf16 x, grad_y in; int8 + fp32 scales out",
+                       "io": "bf16 x, grad_y in; " + {"int8": "int8", "e4m3": "fp8 e4m3"}[fmt[0]]
+                             + " codes + " + fmt[1] + " scales out, y_s_t " + fmt[2],
                        "parallelism": f"replicas x{world} (no exchange)",
                        "l2": f"inputs+outputs rotate over {nsets} buffer sets (>= 3x L2)",
                        "timing": "K calls replayed from CUDA graphs, CUDA events"},
@@ -416,6 +457,8 @@ def run_sdq(args):
         }
         if per is not None:
             line["per_workload"] = per
+        if per_fmt is not None:
+            line["per_format"] = per_fmt
         print(json.dumps(line), flush=True)
     import torch.distributed as tdist
     if tdist.is_initialized():

@@ -155,11 +155,12 @@ class Workload:
     def Kg(self) -> int:
         return self.K // self.group_size
 
-    def algorithmic_bytes(self) -> int:
+    def algorithmic_bytes(self, scale_bytes: int = 4) -> int:
         """Bytes any fused implementation must move: read x and grad_y (6 B per
-        (m, k)), write grad_input_q (2 B) and y_q_t (1 B), plus the fp32 scales."""
+        (m, k)), write grad_input_q (2 B) and y_q_t (1 B) codes, plus the
+        scales (fp32: 4 B each; E8M0: 1 B)."""
         mk = self.M * self.K
-        return 6 * mk + 3 * mk + 4 * self.M * 2 * self.Kg + 4 * self.K * self.Mg
+        return 6 * mk + 3 * mk + scale_bytes * (self.M * 2 * self.Kg + self.K * self.Mg)
 
     def describe(self) -> Dict[str, object]:
         return {"workload": self.name, "M": self.M, "K": self.K,
