@@ -32,10 +32,11 @@ __all__ = [
     "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
     "sdq_fuse_host_workspace_bytes", "sdq_validate",
     "sdq_device_status", "SdqError", "Status", "status_string", "last_cuda_error", "version",
-    "LIB_PATH", "GROUP_SIZE",
+    "LIB_PATH", "GROUP_SIZE", "GROUP_SIZES",
 ]
 
 GROUP_SIZE = 128
+GROUP_SIZES = (32, 64, 128)   # the kernel's tile (128 x 128) holds whole groups of these sizes
 
 
 _E8M0_DTYPES = tuple(d for d in (torch.uint8, getattr(torch, "float8_e8m0fnu", None)) if d is not None)
@@ -95,8 +96,10 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", s
         raise ValueError(f"grad_y shape {tuple(grad_y.shape)} != {(M, K)}")
     if x.dtype != torch.bfloat16 or grad_y.dtype != torch.bfloat16:
         raise ValueError("x and grad_y must be bfloat16")
-    if group_size != GROUP_SIZE or K % group_size:
-        raise ValueError(f"group_size must be 128 and K={K} a multiple of it")
+    if group_size not in GROUP_SIZES or K % GROUP_SIZE:
+        raise ValueError(f"group_size must be one of {GROUP_SIZES} and K={K} a multiple of 128")
+    if not want_cuda and group_size != GROUP_SIZE:
+        raise ValueError("the host-buffer entry points take group_size 128 only")
     names = ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")
     dtypes = (_CODE_DTYPES[codes], _SCALE_DTYPES[scales]) * 2
     for name, t, shape, dts in zip(names, outs, output_shapes(M, K, group_size, y_scale_layout), dtypes):

@@ -24,17 +24,37 @@ constexpr int kStages = SDQ_STAGES;
 
 constexpr int kMaxDevices = 64;
 
-// One kernel per output format (SDQ_FMT_* bits 0..2).
+// One kernel per group size (32, 64, 128) and output format (SDQ_FMT_* bits 0..2).
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const sdq::Params);
 constexpr int kFormats = 8;
-KernelFn kernel_for(uint32_t format) {
-  static constexpr KernelFn table[kFormats] = {
-      sdq::fuse_kernel<kStages, false, false, false>, sdq::fuse_kernel<kStages, true, false, false>,
-      sdq::fuse_kernel<kStages, false, true, false>,  sdq::fuse_kernel<kStages, true, true, false>,
-      sdq::fuse_kernel<kStages, false, false, true>,  sdq::fuse_kernel<kStages, true, false, true>,
-      sdq::fuse_kernel<kStages, false, true, true>,   sdq::fuse_kernel<kStages, true, true, true>};
-  return table[format & (kFormats - 1)];
+constexpr int kKernels = 3 * kFormats;
+
+template <int G>
+constexpr KernelFn kernel_of(int f) {
+  switch (f) {
+    case 0: return sdq::fuse_kernel<kStages, G, false, false, false>;
+    case 1: return sdq::fuse_kernel<kStages, G, true, false, false>;
+    case 2: return sdq::fuse_kernel<kStages, G, false, true, false>;
+    case 3: return sdq::fuse_kernel<kStages, G, true, true, false>;
+    case 4: return sdq::fuse_kernel<kStages, G, false, false, true>;
+    case 5: return sdq::fuse_kernel<kStages, G, true, false, true>;
+    case 6: return sdq::fuse_kernel<kStages, G, false, true, true>;
+    default: return sdq::fuse_kernel<kStages, G, true, true, true>;
+  }
 }
+
+// Kernel number n = 8 * (0, 1, 2 for group size 32, 64, 128) + format bits.
+KernelFn kernel_at(int n) {
+  const int f = n % kFormats;
+  return n < kFormats ? kernel_of<32>(f) : n < 2 * kFormats ? kernel_of<64>(f) : kernel_of<128>(f);
+}
+
+KernelFn kernel_for(int32_t group_size, uint32_t format) {
+  const int gi = group_size == 32 ? 0 : group_size == 64 ? 1 : 2;
+  return kernel_at(gi * kFormats + static_cast<int>(format & (kFormats - 1)));
+}
+
+bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE; }
 thread_local int t_last_cuda_error = 0;
 
 int cuda_fail(cudaError_t e) {
@@ -86,8 +106,8 @@ int current_device(DeviceState** out) {
   DeviceState& d = g_dev[dev];
   std::call_once(d.init, [&d, dev] {
     d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-    for (int f = 0; f < kFormats; ++f) {
-      const auto kernel = kernel_for(static_cast<uint32_t>(f));
+    for (int n = 0; n < kKernels; ++n) {
+      const auto kernel = kernel_at(n);
       if (d.init_err == cudaSuccess)
         d.init_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(sdq::smem_bytes<kStages>()));
@@ -122,7 +142,8 @@ int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
 // `limit_ns` = 0: the default wait limit; `withhold` = 1 only for the
 // failure-path test hook.
 int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void* yst, int64_t M,
-           int64_t K, uint32_t format, cudaStream_t stream, uint64_t limit_ns = 0, int withhold = 0) {
+           int64_t K, int32_t group_size, uint32_t format, cudaStream_t stream,
+           uint64_t limit_ns = 0, int withhold = 0) {
   DeviceState* d = nullptr;
   int st = current_device(&d);
   if (st != SDQ_OK) return st;
@@ -138,6 +159,8 @@ int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void*
   p.K = static_cast<int32_t>(K);
   p.Kg = static_cast<int32_t>(K / sdq::kG);
   p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
+  p.gis_cols = static_cast<int32_t>(2 * K / group_size);
+  p.ys_groups = static_cast<int32_t>((M + group_size - 1) / group_size);
   p.num_tiles = p.Mg * p.Kg;
   p.yqt_vec16 = (M % 16 == 0) ? 1 : 0;
   p.wait_limit_ns = limit_ns ? limit_ns : wait_limit_ns();
@@ -156,7 +179,7 @@ int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void*
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(format), mx, mg, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format), mx, mg, p);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -204,7 +227,7 @@ const char* sdq_status_string(int status) {
   switch (status) {
     case SDQ_OK: return "SDQ_OK";
     case SDQ_ERR_NULL: return "SDQ_ERR_NULL: a required pointer is NULL";
-    case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 128";
+    case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 32, 64 or 128 (128 for the host-buffer entry points)";
     case SDQ_ERR_SHAPE: return "SDQ_ERR_SHAPE: need M >= 0 and K a positive multiple of 128 within the size limits";
     case SDQ_ERR_ALIGN: return "SDQ_ERR_ALIGN: x, grad_y, grad_input_q, y_q_t need 16-byte and scales 4-byte alignment";
     case SDQ_ERR_CUDA: return "SDQ_ERR_CUDA: a CUDA call failed (see sdq_last_cuda_error)";
@@ -221,7 +244,7 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
                         int64_t K, int32_t group_size, uint32_t format) {
   if (format & ~static_cast<uint32_t>(SDQ_FMT_E4M3 | SDQ_FMT_E8M0 | SDQ_FMT_YS_MG_K))
     return SDQ_ERR_FORMAT;
-  if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
+  if (!group_size_supported(group_size)) return SDQ_ERR_GROUP;
   if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
     return SDQ_ERR_SHAPE;
   const int64_t tiles = ((M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE) * (K / SDQ_GROUP_SIZE);
@@ -247,7 +270,7 @@ int sdq_fuse_format(const void* x, const void* grad_y, void* grad_input_q, void*
   const int st = sdq_validate_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                                      group_size, format);
   if (st != SDQ_OK || M == 0) return st;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, format,
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, format,
                 static_cast<cudaStream_t>(stream));
 }
 
@@ -326,7 +349,7 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
     // kernel on the caller's stream
     SDQ_CHECK(cudaStreamWaitEvent(cs, d->in_ready[b], 0));
     st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt, base + L.yst, mc,
-                K, 0, cs);
+                K, SDQ_GROUP_SIZE, 0, cs);
     if (st != SDQ_OK) return st;
     SDQ_CHECK(cudaEventRecord(d->out_ready[b], cs));
     // device -> host
@@ -418,7 +441,7 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
                              cudaMemcpyHostToDevice, cs)) != cudaSuccess)
       return cuda_fail(e);
     const int st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt,
-                          base + L.yst, mc, K, 0, cs);
+                          base + L.yst, mc, K, SDQ_GROUP_SIZE, 0, cs);
     if (st != SDQ_OK) return st;
     if ((e = cudaMemcpyAsync(grad_input_q + m0 * 2 * K, base + L.giq, size_t(mc) * 2 * K,
                              cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
@@ -443,7 +466,7 @@ int sdq_fuse_test_stall(const void* x, const void* grad_y, int8_t* grad_input_q,
   const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
   if (st != SDQ_OK || M == 0) return st;
   if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000) return SDQ_ERR_SHAPE;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, 0,
+  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, 0,
                 static_cast<cudaStream_t>(stream), static_cast<uint64_t>(wait_limit_ns), 1);
 }
 

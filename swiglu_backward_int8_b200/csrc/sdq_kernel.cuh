@@ -84,7 +84,9 @@ struct Params {
   void* yst;     // [K, Mg] or [Mg, K], fp32 or E8M0 bytes
   int64_t M;
   int32_t K;
-  int32_t Kg;
+  int32_t Kg;        // 128-channel tiles per row
+  int32_t gis_cols;  // 2K / group size: columns of grad_input_s
+  int32_t ys_groups; // ceil(M / group size): token groups of y_s_t
   int32_t Mg;
   int32_t num_tiles;
   int32_t yqt_vec16;  // M % 16 == 0: y_q_t rows take 16-byte stores
@@ -334,11 +336,24 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uin
   return true;
 }
 
+// Quantization groups of kGS = 32, 64 or 128 elements: a 128 x 128 tile holds
+// 128/kGS groups along each axis, and since a row-pass lane holds 16
+// consecutive channels of a row and a column-pass thread 16 consecutive
+// tokens of a channel pair, a group is kGS/16 neighbouring lanes (threads):
+// its amax takes log2(kGS/16) shuffle steps.
+template <int kGS>
+__device__ __forceinline__ uint32_t group_amax(uint32_t m) {
+  static_assert(kGS == 32 || kGS == 64 || kGS == 128, "group size 32, 64 or 128");
+#pragma unroll
+  for (int o = 1; o < kGS / 16; o <<= 1) m = absmax_bf16x2(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
 // Column pass of one tile: this thread's channels 2cp, 2cp+1 and tokens
-// 16kc .. 16kc+15 of the bf16 y tile -> column amax over the 8 threads that
-// share the channels, the two column scales, codes, two 16-byte pieces of
-// y_q_t rows.
-template <bool kE4M3, bool kE8M0, bool kYsMgK>
+// 16kc .. 16kc+15 of the bf16 y tile -> column amax over the kGS/16 threads
+// that share the channels and the token group, the two column scales, codes,
+// two 16-byte pieces of y_q_t rows.
+template <int kGS, bool kE4M3, bool kE8M0, bool kYsMgK>
 __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab, const Params& p,
                                             int i, int j, int64_t row0, int valid, int cp, int kc) {
   constexpr unsigned kFull = 0xffffffffu;
@@ -349,17 +364,21 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   uint32_t m = absmax_bf16x2(v[0], v[1]);
 #pragma unroll
   for (int tt = 2; tt < 16; ++tt) m = absmax_bf16x2(m, v[tt]);
-  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 1));
-  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 2));
-  m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 4));
-  m &= 0x7FFF7FFFu;
+  m = group_amax<kGS>(m) & 0x7FFF7FFFu;
   float s_lo, i_lo, s_hi, i_hi;
   group_scale<kE4M3, kE8M0>(m & 0xFFFFu, tab, s_lo, i_lo);
   group_scale<kE4M3, kE8M0>(m >> 16, tab, s_hi, i_hi);
   const int ch = j * kG + 2 * cp;
-  if (kc < 2)
-    store_scale<kE8M0>(p.yst, kYsMgK ? int64_t(i) * p.K + ch + kc : int64_t(ch + kc) * p.Mg + i,
-                       kc ? s_hi : s_lo);
+  // the first two threads of each token group store its low / high channel
+  // scale, for the groups that hold a token (a tail tile's later groups don't)
+  constexpr int kTpg = kGS / 16;   // threads per token group
+  const int gk = kc & (kTpg - 1);
+  const int tg = kc / kTpg;        // token group within the tile
+  if (gk < 2 && tg * kGS < valid) {
+    const int64_t grp = int64_t(i) * (kG / kGS) + tg;
+    store_scale<kE8M0>(p.yst, kYsMgK ? grp * p.K + ch + gk : int64_t(ch + gk) * p.ys_groups + grp,
+                       gk ? s_hi : s_lo);
+  }
   uint4 lo, hi;
   if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
     // pre-multiply only the tiny channels; the others use factor 1
@@ -377,7 +396,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   }
 }
 
-template <int STAGES, bool kE4M3, bool kE8M0, bool kYsMgK>
+template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK>
 __global__ void __launch_bounds__(kThreads, 1)
     fuse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy,
                 const Params p) {
@@ -453,7 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* yt = s.ytile[yb];
     // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
     int8_t* giq_t = p.giq + row0 * (2 * int64_t(K)) + j * kG;
-    const int64_t gis_t = row0 * (2 * Kg) + j;   // scale index of (row0, group j)
+    // scale index of (row0, the tile's first d_gate group)
+    const int64_t gis_t = row0 * p.gis_cols + j * (kG / kGS);
 
     // ================= row pass over the tile's two stages
 #pragma unroll
@@ -522,10 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         b = absmax_bf16x2(b, dup[c]);
       }
       uint32_t pr = absmax_bf16x2(__byte_perm(a, b, 0x1054), __byte_perm(a, b, 0x3276));
-      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 1));
-      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 2));
-      pr = absmax_bf16x2(pr, __shfl_xor_sync(kFull, pr, 4));
-      pr &= 0x7FFF7FFFu;
+      pr = group_amax<kGS>(pr) & 0x7FFF7FFFu;
 
       // ---- the row's two scales, computed by each of its 8 lanes (no shuffles
       // on this path); lanes 0 and 1 of the row store them
@@ -533,8 +550,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       group_scale<kE4M3, kE8M0>(pr >> 16, tab, sg, ig);
       group_scale<kE4M3, kE8M0>(pr & 0xFFFFu, tab, su, iu);
       const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
-      if (cq < 2 && rbase + rr < valid)
-        store_scale<kE8M0>(p.gis, gis_t + (rbase + rr) * (2 * Kg) + cq * Kg, cq ? su : sg);
+      // the first two lanes of each channel group store its d_gate / d_up
+      // scale (the d_up groups start at column gis_cols / 2)
+      {
+        constexpr int kLpg = kGS / 16;   // lanes per channel group
+        const int gl = cq & (kLpg - 1);
+        if (gl < 2 && rbase + rr < valid)
+          store_scale<kE8M0>(p.gis, gis_t + int64_t(rbase + rr) * p.gis_cols + cq / kLpg +
+                                        gl * (p.gis_cols >> 1),
+                             gl ? su : sg);
+      }
 
       // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
       const int r = rbase + rr;   // this lane's row within the tile
@@ -563,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[pb]), ((k - 1) / kYBuf) & 1, lim,
                                            abort_flag));
       if (!ok) break;
-      column_pass<kE4M3, kE8M0, kYsMgK>(s.ytile[pb], tab, p, pi, pj, prow0, pvalid, cp, kc);
+      column_pass<kGS, kE4M3, kE8M0, kYsMgK>(s.ytile[pb], tab, p, pi, pj, prow0, pvalid, cp, kc);
       mbar_arrive(smem_u32(&s.y_free[pb]));
     }
     pi = i;
@@ -577,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k = my_tiles - 1;
     ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready[k % kYBuf]), (k / kYBuf) & 1, lim,
                                          abort_flag));
-    if (ok) column_pass<kE4M3, kE8M0, kYsMgK>(s.ytile[k % kYBuf], tab, p, pi, pj, prow0, pvalid, cp, kc);
+    if (ok) column_pass<kGS, kE4M3, kE8M0, kYsMgK>(s.ytile[k % kYBuf], tab, p, pi, pj, prow0, pvalid, cp, kc);
   }
 
   __syncthreads();   // every thread arrives here, whether it stopped early or not

@@ -154,21 +154,22 @@ def _e4m3_values():
 E4M3_VALUE = _e4m3_values()
 
 
-def run_cuda_fmt(x_u16: np.ndarray, gy_u16: np.ndarray, codes: int, scales: int, ys_layout: int):
+def run_cuda_fmt(x_u16: np.ndarray, gy_u16: np.ndarray, codes: int, scales: int, ys_layout: int,
+                 group_size: int = 128):
     """The device entry point in a chosen format, on guarded outputs; returns
     numpy (code bytes, scales, code bytes, scales) like the format oracle."""
     import swiglu_backward_int8_b200 as sdq
     M, K = gy_u16.shape
     x = to_device_bf16(x_u16)
     gy = to_device_bf16(gy_u16)
-    shp = oracle.output_shapes_fmt(M, K, 128, ys_layout)
+    shp = oracle.output_shapes_fmt(M, K, group_size, ys_layout)
     sq = SENTINEL_CODE[codes]
     mk_s = (lambda s: Guarded(s, torch.uint8, SENTINEL_E8M0)) if scales else \
         (lambda s: Guarded(s, torch.float32, float("nan")))
     outs = [Guarded(shp[0], torch.uint8, sq), mk_s(shp[1]), Guarded(shp[2], torch.uint8, sq), mk_s(shp[3])]
     fmt = (sdq.FMT_E4M3 if codes else 0) | (sdq.FMT_E8M0 if scales else 0) | \
         (sdq.FMT_YS_MG_K if ys_layout else 0)
-    sdq.sdq_fuse_format(x.data_ptr(), gy.data_ptr(), *(o.t.data_ptr() for o in outs), M, K, 128, fmt,
+    sdq.sdq_fuse_format(x.data_ptr(), gy.data_ptr(), *(o.t.data_ptr() for o in outs), M, K, group_size, fmt,
                         torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert sdq.sdq_device_status() == 0
@@ -198,7 +199,7 @@ def _scale_values(s, scales):
     return np.ldexp(1.0, s.astype(np.int64) - 127) if scales else s.astype(np.float64)
 
 
-def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where=""):
+def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", group_size: int = 128):
     """Assert the format tolerances; returns mismatch statistics."""
     giq, gis, yqt, yst = got
     rq, rs, ryq, rys = ref
@@ -216,7 +217,7 @@ def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where=""):
         else:
             rel = np.abs(a.astype(np.float64) - b.astype(np.float64)) / np.abs(b.astype(np.float64))
             assert rel.max(initial=0) <= SCALE_MAX_REL, f"{where} {name}: max rel = {rel.max()}"
-    G = 128
+    G = group_size
     M = giq.shape[0]
     for name, a, b, sa, sb in (("grad_input_q", giq, rq, np.repeat(gis, G, axis=1), np.repeat(rs, G, axis=1)),
                                ("y_q_t", yqt, ryq, np.repeat(yst, G, axis=1)[:, :M],

@@ -50,7 +50,11 @@ A = 1 << 20  # a 16-byte-aligned fake address: validation never dereferences
 
 @pytest.mark.parametrize("args,status", [
     (dict(), 0),
-    (dict(group_size=64), 2),
+    (dict(group_size=64), 0),
+    (dict(group_size=32), 0),
+    (dict(group_size=96), 2),
+    (dict(group_size=256), 2),
+    (dict(group_size=64, K=192), 3),      # the tile stays 128 channels wide
     (dict(K=100), 3),
     (dict(K=0), 3),
     (dict(M=-1), 3),
@@ -80,7 +84,7 @@ def test_fuse_rejects_before_any_cuda_call():
         sdq.sdq_fuse(A, A, A, A, A, A, 256, 200, 128)
     assert ei.value.status == sdq.Status.ERR_SHAPE
     with pytest.raises(sdq.SdqError) as ei:
-        sdq.sdq_fuse(A, A, A, A, A, A, 256, 256, 32)
+        sdq.sdq_fuse(A, A, A, A, A, A, 256, 256, 16)
     assert ei.value.status == sdq.Status.ERR_GROUP
     sdq.sdq_fuse(0, 0, 0, 0, 0, 0, 0, 256, 128)  # M == 0: nothing to do
 
@@ -119,7 +123,8 @@ def test_torch_wrapper_argument_checks():
     (0, dict(grad_input_s=A + 1), 4),
     (1, dict(y_s_t=A + 2), 4),             # E4M3 codes with fp32 scales: 4-byte scales
     (6, dict(grad_input_q=A + 1), 4),      # code arrays stay 16-byte aligned
-    (3, dict(group_size=64), 2),
+    (3, dict(group_size=48), 2),
+    (3, dict(group_size=32), 0),
     (5, dict(M=0, x=0), 0),
 ])
 def test_validate_format_statuses(fmt, args, status):

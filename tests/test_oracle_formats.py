@@ -214,24 +214,28 @@ def test_whole_op_fmt_ys_layouts_transpose(codes, scales):
         assert np.array_equal(u, v)
 
 
+@pytest.mark.parametrize("G", [128, 64, 32])
 @pytest.mark.parametrize("codes,scales", FORMATS)
-def test_whole_op_fmt_groups_relate_to_stage1(codes, scales):
+def test_whole_op_fmt_groups_relate_to_stage1(codes, scales, G):
     # every group of all four outputs equals the exact restatement of the
-    # format applied to that group's bf16 intermediates (M = 40: one tail group)
-    w = W.small_workload(40, 256, seed=6)
+    # format applied to that group's bf16 intermediates (M = 40: a tail group)
+    M, K = 40, 256
+    w = W.small_workload(M, K, seed=6)
     x, gy = W.make_inputs(w)
-    giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, 128, codes, scales, 0)
+    giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, G, codes, scales, 0)
+    assert gis.shape == (M, 2 * K // G) and yst.shape == (K, (M + G - 1) // G)
     y, dg, du = oracle.swiglu_bwd_bf16(x, gy)
     V = np.concatenate([dg, du], axis=1)
-    for m in range(0, 40, 3):
-        for j in range(4):
-            want_q, want_s = _expected_group(V[m, j * 128:(j + 1) * 128], codes, scales)
-            assert list(giq[m, j * 128:(j + 1) * 128]) == want_q
+    for m in range(0, M, 3):
+        for j in range(2 * K // G):
+            want_q, want_s = _expected_group(V[m, j * G:(j + 1) * G], codes, scales)
+            assert list(giq[m, j * G:(j + 1) * G]) == want_q
             assert gis[m, j] == want_s
-    for k in range(0, 256, 5):
-        want_q, want_s = _expected_group(y[:, k], codes, scales)
-        assert list(yqt[k, :]) == want_q
-        assert yst[k, 0] == want_s
+    for k in range(0, K, 5):
+        for i in range((M + G - 1) // G):
+            want_q, want_s = _expected_group(y[i * G:(i + 1) * G, k], codes, scales)
+            assert list(yqt[k, i * G:(i + 1) * G]) == want_q
+            assert yst[k, i] == want_s
 
 
 def test_whole_op_e4m3_gate32_closed_form():

@@ -278,14 +278,16 @@ def _gate32_case(M, K):
     return f64_to_bf16_bits(x), f64_to_bf16_bits(gy), a, w, e
 
 
-@pytest.mark.parametrize("M,K", [(200, 256), (7, 128), (129, 384)])
-def test_whole_op_gate32_closed_form(M, K):
+@pytest.mark.parametrize("M,K,G", [(200, 256, 128), (7, 128, 128), (129, 384, 128),
+                                   (200, 256, 64), (129, 128, 32)])
+def test_whole_op_gate32_closed_form(M, K, G):
     x, gy, a, w, e = _gate32_case(M, K)
-    giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy)
-    G, Kg, Mg = 128, K // 128, (M + 127) // 128
+    giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, G)
+    Kg, Mg = K // G, (M + G - 1) // G
     f32 = np.float32
-    # d_gate groups: amax over a 128-channel group = 7 * a(m) * 2^-e (w cycles 1,3,5,7)
-    # -> q = round(w * 127 / 7) = 18, 54, 91, 127 (no value near a half).
+    # d_gate groups: amax over a G-channel group (G >= 32 holds the whole cycle
+    # w = 1, 3, 5, 7) = 7 * a(m) * 2^-e -> q = round(w * 127 / 7) = 18, 54, 91, 127
+    # (no value near a half).
     q_dg = {1: 18, 3: 54, 5: 91, 7: 127}
     for m in range(M):
         s_dg = f32(f32(7 * a[m] * 2.0 ** -e[m]) / f32(127))
@@ -305,7 +307,7 @@ def test_whole_op_gate32_closed_form(M, K):
         if amax_a == 8:
             want = np.array([q_y[int(t)] for t in a[t0:t1]], np.int8)
             assert np.all(yqt[:, t0:t1] == want[None, :])
-    assert yqt.shape == (K, M) and yst.shape == (K, Mg)
+    assert yqt.shape == (K, M) and yst.shape == (K, Mg) and gis.shape == (M, 2 * Kg)
 
 
 def test_whole_op_gate_zero_closed_form():
