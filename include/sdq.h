@@ -67,7 +67,9 @@ typedef enum sdq_status {
   SDQ_ERR_TIMEOUT = 6,   /* a device-side wait hit its time limit (sdq_device_status) */
   SDQ_ERR_WORKSPACE = 7, /* the workspace given to sdq_fuse_host is too small        */
   SDQ_ERR_TOO_LARGE = 8, /* sdq_fuse_host_noalloc: K too large for its fixed scratch  */
-  SDQ_ERR_FORMAT = 9     /* sdq_fuse_format: unknown bits in `format`                */
+  SDQ_ERR_FORMAT = 9,    /* sdq_fuse_format: unknown bits in `format`                */
+  SDQ_ERR_STRIDE = 10    /* sdq_fuse_strided: a leading dimension below its row length
+                            or above SDQ_MAX_LD                                      */
 } sdq_status;
 
 /* Largest accepted sizes: M < 2^31 (tensor-map coordinates are 32-bit) and
@@ -75,6 +77,8 @@ typedef enum sdq_status {
 #define SDQ_GROUP_SIZE 128
 #define SDQ_MAX_M 2147483647LL
 #define SDQ_MAX_K 1048576LL
+#define SDQ_MAX_LD (1LL << 36) /* largest leading dimension (tensor-map strides < 2^40 bytes) */
+#define SDQ_MAX_LD_ROWS (1LL << 24) /* largest ld of grad_input_q and grad_input_s     */
 
 /*
  * sdq_fuse -- the op on device buffers.
@@ -148,6 +152,43 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
                         const void* grad_input_s, const void* y_q_t,
                         const void* y_s_t, int64_t M, int64_t K,
                         int32_t group_size, uint32_t format);
+
+/*
+ * sdq_fuse_strided -- sdq_fuse_format on arrays with their own row strides:
+ * each array is row-major with `ld_*` ELEMENTS from the start of one row to
+ * the next (at least the row length; up to SDQ_MAX_LD), and gate and up are
+ * separate [M, K] arrays.  The page's x = [gate | up] is gate = x,
+ * up = x + K (elements), ld_gate = ld_up = 2K; a slice of a wider buffer,
+ * padded rows, or gate and up held apart are all the same call.
+ *   gate, up, grad_y   device, bf16 [M, K] each; 16-byte aligned; ld a
+ *                      multiple of 8 (rows start on 16 bytes)
+ *   grad_input_q       [M, 2K] codes; 16-byte aligned; ld a multiple of 16,
+ *                      at most SDQ_MAX_LD_ROWS
+ *   grad_input_s       [M, 2K/group_size] scales; 2K/group_size <= ld <=
+ *                      SDQ_MAX_LD_ROWS
+ *   y_q_t              [K, M] codes; 16-byte aligned; any ld >= M (a multiple
+ *                      of 16 takes 16-byte stores, others byte stores)
+ *   y_s_t              [K, ceil(M/group_size)] (or [ceil(M/group_size), K]
+ *                      with SDQ_FMT_YS_MG_K) scales
+ *   M, K, group_size, format, stream: as sdq_fuse_format.
+ * Inputs may overlap each other (gate and up often do: two halves of one
+ * buffer); outputs must not overlap inputs or each other.  SDQ_ERR_STRIDE
+ * for a leading dimension out of range, SDQ_ERR_ALIGN for a misaligned one.
+ */
+int sdq_fuse_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                     const void* grad_y, int64_t ld_grad_y, void* grad_input_q,
+                     int64_t ld_grad_input_q, void* grad_input_s, int64_t ld_grad_input_s,
+                     void* y_q_t, int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t,
+                     int64_t M, int64_t K, int32_t group_size, uint32_t format,
+                     void* stream);
+
+/* The argument checks of sdq_fuse_strided alone: no CUDA call, no launch. */
+int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                         const void* grad_y, int64_t ld_grad_y, const void* grad_input_q,
+                         int64_t ld_grad_input_q, const void* grad_input_s,
+                         int64_t ld_grad_input_s, const void* y_q_t, int64_t ld_y_q_t,
+                         const void* y_s_t, int64_t ld_y_s_t, int64_t M, int64_t K,
+                         int32_t group_size, uint32_t format);
 
 /*
  * sdq_fuse_host -- the op on HOST buffers (same shapes and layouts as

@@ -23,11 +23,12 @@ import torch
 
 from ._lib import (FMT_E4M3, FMT_E8M0, FMT_YS_MG_K, LIB_PATH, SdqError, Status, last_cuda_error,
                    sdq_device_status, sdq_fuse, sdq_fuse_format, sdq_fuse_host,
-                   sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_validate,
-                   sdq_validate_format, status_string, version)
+                   sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_fuse_strided,
+                   sdq_validate, sdq_validate_format, sdq_validate_strided, status_string, version)
 
 __all__ = [
-    "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs",
+    "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_split",
+    "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs", "sdq_fuse_strided", "sdq_validate_strided",
     "output_shapes", "output_format", "sdq_fuse", "sdq_fuse_format", "sdq_validate_format",
     "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
     "sdq_fuse_host_workspace_bytes", "sdq_validate",
@@ -84,6 +85,39 @@ def _infer(kind: str, given: Optional[str], t: torch.Tensor, table) -> str:
     return given
 
 
+def _rows(name: str, t: torch.Tensor, shape, dtypes, want_cuda: bool, device) -> int:
+    """Check a 2-D row-major operand (rows may be padded: stride(0) >= its
+    row); returns its leading dimension in elements."""
+    if t.dim() != 2 or tuple(t.shape) != tuple(shape) or t.dtype not in dtypes:
+        raise ValueError(f"{name}: expected {' or '.join(map(str, dtypes))} {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)}")
+    if t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride along its rows")
+    if t.shape[0] > 1 and t.stride(0) < t.shape[1]:
+        raise ValueError(f"{name}: rows overlap (stride {t.stride(0)} < row length {t.shape[1]})")
+    if not want_cuda and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous for the host-buffer entry points")
+    if want_cuda and (not t.is_cuda or t.device != device):
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if not want_cuda and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    return int(t.stride(0)) if t.shape[0] > 1 else int(t.shape[1])
+
+
+def _check_group(K: int, group_size: int, want_cuda: bool):
+    if group_size not in GROUP_SIZES or K % GROUP_SIZE:
+        raise ValueError(f"group_size must be one of {GROUP_SIZES} and K={K} a multiple of 128")
+    if not want_cuda and group_size != GROUP_SIZE:
+        raise ValueError("the host-buffer entry points take group_size 128 only")
+
+
+def _check_outputs(M, K, outs, group_size, want_cuda, codes, scales, y_scale_layout, device):
+    names = ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")
+    dtypes = (_CODE_DTYPES[codes], _SCALE_DTYPES[scales]) * 2
+    return [_rows(n, t, shp, dts, want_cuda, device)
+            for n, t, shp, dts in zip(names, outs, output_shapes(M, K, group_size, y_scale_layout), dtypes)]
+
+
 def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", scales="fp32",
                    y_scale_layout="k_mg"):
     if x.dim() != 2 or grad_y.dim() != 2:
@@ -92,28 +126,21 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", s
     if K2 % 2:
         raise ValueError(f"x has an odd channel count {K2}; expected [gate | up]")
     K = K2 // 2
-    if tuple(grad_y.shape) != (M, K):
-        raise ValueError(f"grad_y shape {tuple(grad_y.shape)} != {(M, K)}")
-    if x.dtype != torch.bfloat16 or grad_y.dtype != torch.bfloat16:
-        raise ValueError("x and grad_y must be bfloat16")
-    if group_size not in GROUP_SIZES or K % GROUP_SIZE:
-        raise ValueError(f"group_size must be one of {GROUP_SIZES} and K={K} a multiple of 128")
-    if not want_cuda and group_size != GROUP_SIZE:
-        raise ValueError("the host-buffer entry points take group_size 128 only")
-    names = ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")
-    dtypes = (_CODE_DTYPES[codes], _SCALE_DTYPES[scales]) * 2
-    for name, t, shape, dts in zip(names, outs, output_shapes(M, K, group_size, y_scale_layout), dtypes):
-        if tuple(t.shape) != shape or t.dtype not in dts:
-            raise ValueError(f"{name}: expected {' or '.join(map(str, dts))} {shape}, "
-                             f"got {t.dtype} {tuple(t.shape)}")
-    for name, t in zip(("x", "grad_y") + names, (x, grad_y) + tuple(outs)):
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous")
-        if want_cuda and (not t.is_cuda or t.device != x.device):
-            raise ValueError(f"{name} must be a CUDA tensor on {x.device}")
-        if not want_cuda and t.is_cuda:
-            raise ValueError(f"{name} must be a host tensor")
-    return M, K
+    _check_group(K, group_size, want_cuda)
+    bf16 = (torch.bfloat16,)
+    ld_x = _rows("x", x, (M, 2 * K), bf16, want_cuda, x.device)
+    ld_gy = _rows("grad_y", grad_y, (M, K), bf16, want_cuda, x.device)
+    lds = _check_outputs(M, K, outs, group_size, want_cuda, codes, scales, y_scale_layout, x.device)
+    return M, K, ld_x, ld_gy, lds
+
+
+def _call_strided(gate, ld_gate, up, ld_up, grad_y, ld_gy, outs, lds, M, K, group_size, fmt, device):
+    with torch.cuda.device(device):
+        stream = torch.cuda.current_stream(device).cuda_stream
+        q, s, yq, ys = outs
+        sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y.data_ptr(), ld_gy, q.data_ptr(), lds[0],
+                         s.data_ptr(), lds[1], yq.data_ptr(), lds[2], ys.data_ptr(), lds[3], M, K,
+                         group_size, fmt, stream)
 
 
 def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_input_q: torch.Tensor,
@@ -125,18 +152,44 @@ def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_inpu
     current CUDA stream of x's device.  The code format ("int8" or "e4m3")
     and the scale format ("fp32" or "e8m0") follow the dtypes of
     grad_input_q and grad_input_s unless given; ``y_scale_layout`` is "k_mg"
-    (y_s_t [K, ceil(M/128)]) or "mg_k".  Raises ValueError on bad arguments
-    and SdqError on a library status."""
+    (y_s_t [K, ceil(M/G)]) or "mg_k"; ``group_size`` is 128, 64 or 32.  Every
+    tensor is 2-D row-major; rows may be padded (a slice of a wider buffer):
+    the library takes each tensor's row stride.  Raises ValueError on bad
+    arguments and SdqError on a library status."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
     codes = _infer("codes", codes, grad_input_q, _CODE_DTYPES)
     scales = _infer("scales", scales, grad_input_s, _SCALE_DTYPES)
     fmt = output_format(codes, scales, y_scale_layout)
-    M, K = _check_tensors(x, grad_y, outs, group_size, True, codes, scales, y_scale_layout)
-    with torch.cuda.device(x.device):
-        stream = torch.cuda.current_stream(x.device).cuda_stream
-        sdq_fuse_format(x.data_ptr(), grad_y.data_ptr(), grad_input_q.data_ptr(),
-                        grad_input_s.data_ptr(), y_q_t.data_ptr(), y_s_t.data_ptr(), M, K,
-                        group_size, fmt, stream)
+    M, K, ld_x, ld_gy, lds = _check_tensors(x, grad_y, outs, group_size, True, codes, scales,
+                                            y_scale_layout)
+    _call_strided(x.data_ptr(), ld_x, x.data_ptr() + 2 * K, ld_x, grad_y, ld_gy, outs, lds, M, K,
+                  group_size, fmt, x.device)
+
+
+def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad_y: torch.Tensor,
+                                      grad_input_q: torch.Tensor, grad_input_s: torch.Tensor,
+                                      y_q_t: torch.Tensor, y_s_t: torch.Tensor,
+                                      group_size: int = GROUP_SIZE, *, codes: Optional[str] = None,
+                                      scales: Optional[str] = None,
+                                      y_scale_layout: str = "k_mg") -> None:
+    """The op with gate and up as two [M, K] bf16 tensors instead of one
+    x = [gate | up] (e.g. the two halves of a fused projection kept apart);
+    otherwise as silu_dot_fwd_bwd_quant_fuse."""
+    outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
+    codes = _infer("codes", codes, grad_input_q, _CODE_DTYPES)
+    scales = _infer("scales", scales, grad_input_s, _SCALE_DTYPES)
+    fmt = output_format(codes, scales, y_scale_layout)
+    if gate.dim() != 2:
+        raise ValueError("gate must be 2-D")
+    M, K = gate.shape
+    _check_group(K, group_size, True)
+    bf16 = (torch.bfloat16,)
+    ld_g = _rows("gate", gate, (M, K), bf16, True, gate.device)
+    ld_u = _rows("up", up, (M, K), bf16, True, gate.device)
+    ld_gy = _rows("grad_y", grad_y, (M, K), bf16, True, gate.device)
+    lds = _check_outputs(M, K, outs, group_size, True, codes, scales, y_scale_layout, gate.device)
+    _call_strided(gate.data_ptr(), ld_g, up.data_ptr(), ld_u, grad_y, ld_gy, outs, lds, M, K,
+                  group_size, fmt, gate.device)
 
 
 def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
@@ -149,7 +202,7 @@ def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
     device ``workspace`` (uint8 CUDA tensor of at least
     ``sdq_fuse_host_workspace_bytes(M, K, chunk_rows)`` bytes)."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
-    M, K = _check_tensors(x, grad_y, outs, group_size, want_cuda=False)
+    M, K, _, _, _ = _check_tensors(x, grad_y, outs, group_size, want_cuda=False)
     if not workspace.is_cuda:
         raise ValueError("workspace must be a CUDA tensor")
     dev = device or workspace.device

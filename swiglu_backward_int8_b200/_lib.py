@@ -32,6 +32,11 @@ _lib.sdq_fuse_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctype
 _lib.sdq_fuse_format.restype = ctypes.c_int
 _lib.sdq_validate_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctypes.c_uint32]
 _lib.sdq_validate_format.restype = ctypes.c_int
+_STRIDED = [_P, _I64] * 7 + [_I64, _I64, _I32, ctypes.c_uint32]
+_lib.sdq_fuse_strided.argtypes = _STRIDED + [_P]
+_lib.sdq_fuse_strided.restype = ctypes.c_int
+_lib.sdq_validate_strided.argtypes = _STRIDED
+_lib.sdq_validate_strided.restype = ctypes.c_int
 _lib.sdq_fuse_host.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P, ctypes.c_size_t, _I64, _P]
 _lib.sdq_fuse_host.restype = ctypes.c_int
 _lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
@@ -61,6 +66,7 @@ class Status(enum.IntEnum):
     ERR_WORKSPACE = 7
     ERR_TOO_LARGE = 8
     ERR_FORMAT = 9
+    ERR_STRIDE = 10
 
 
 # Output-format bits of sdq_fuse_format (include/sdq.h): 0 = INT8 codes, fp32
@@ -111,6 +117,27 @@ def sdq_fuse_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y
     """Raw-pointer form of the device entry point with an output format (FMT_* bits)."""
     _check(_lib.sdq_fuse_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                                 group_size, format, stream or 0), "sdq_fuse_format")
+
+
+def sdq_fuse_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: int, ld_grad_y: int,
+                     grad_input_q: int, ld_grad_input_q: int, grad_input_s: int, ld_grad_input_s: int,
+                     y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int, M: int, K: int,
+                     group_size: int = 128, format: int = 0, stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the strided entry point (leading dimensions in elements)."""
+    _check(_lib.sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
+                                 ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t,
+                                 y_s_t, ld_y_s_t, M, K, group_size, format, stream or 0),
+           "sdq_fuse_strided")
+
+
+def sdq_validate_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: int, ld_grad_y: int,
+                         grad_input_q: int, ld_grad_input_q: int, grad_input_s: int,
+                         ld_grad_input_s: int, y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int,
+                         M: int, K: int, group_size: int = 128, format: int = 0) -> int:
+    """Argument checks of sdq_fuse_strided only (no CUDA call); returns the status code."""
+    return int(_lib.sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
+                                         ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t,
+                                         ld_y_q_t, y_s_t, ld_y_s_t, M, K, group_size, format))
 
 
 def sdq_validate_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,

@@ -25,7 +25,7 @@ constexpr int kStages = SDQ_STAGES;
 constexpr int kMaxDevices = 64;
 
 // One kernel per group size (32, 64, 128) and output format (SDQ_FMT_* bits 0..2).
-using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const sdq::Params);
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const sdq::Params);
 constexpr int kFormats = 8;
 constexpr int kKernels = 3 * kFormats;
 
@@ -138,31 +138,69 @@ int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
   return SDQ_OK;
 }
 
+// One call's arrays and leading dimensions (elements from one row to the
+// next), as sdq_fuse_strided takes them.
+struct Arrays {
+  const void* gate; int64_t ld_gate;
+  const void* up;   int64_t ld_up;
+  const void* gy;   int64_t ld_gy;
+  void* giq; int64_t ld_giq;
+  void* gis; int64_t ld_gis;
+  void* yqt; int64_t ld_yqt;
+  void* yst; int64_t ld_yst;
+};
+
+// Contiguous arrays of the page's layout: x = [gate | up] [M, 2K], grad_y
+// [M, K], the outputs packed.
+Arrays packed(const void* x, const void* gy, void* giq, void* gis, void* yqt, void* yst, int64_t M,
+              int64_t K, int32_t group_size, uint32_t format) {
+  const int64_t gsz = group_size > 0 ? group_size : 1;
+  Arrays a;
+  a.gate = x;
+  a.ld_gate = 2 * K;
+  a.up = x ? static_cast<const uint8_t*>(x) + 2 * K : nullptr;   // bf16: K elements on
+  a.ld_up = 2 * K;
+  a.gy = gy;
+  a.ld_gy = K;
+  a.giq = giq;
+  a.ld_giq = 2 * K;
+  a.gis = gis;
+  a.ld_gis = 2 * K / gsz;
+  a.yqt = yqt;
+  a.ld_yqt = M;
+  a.yst = yst;
+  a.ld_yst = (format & SDQ_FMT_YS_MG_K) ? K : (M + gsz - 1) / gsz;
+  return a;
+}
+
 // Launch on validated arguments (M > 0).  `format`: SDQ_FMT_* bits;
 // `limit_ns` = 0: the default wait limit; `withhold` = 1 only for the
 // failure-path test hook.
-int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void* yst, int64_t M,
-           int64_t K, int32_t group_size, uint32_t format, cudaStream_t stream,
-           uint64_t limit_ns = 0, int withhold = 0) {
+int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t format,
+           cudaStream_t stream, uint64_t limit_ns = 0, int withhold = 0) {
   DeviceState* d = nullptr;
   int st = current_device(&d);
   if (st != SDQ_OK) return st;
-  CUtensorMap mx, mg;
-  if ((st = make_map(&mx, x, 2 * K, M, 4 * K)) != SDQ_OK) return st;
-  if ((st = make_map(&mg, gy, K, M, 2 * K)) != SDQ_OK) return st;
+  CUtensorMap mgate, mup, mdy;
+  if ((st = make_map(&mgate, a.gate, K, M, 2 * a.ld_gate)) != SDQ_OK) return st;
+  if ((st = make_map(&mup, a.up, K, M, 2 * a.ld_up)) != SDQ_OK) return st;
+  if ((st = make_map(&mdy, a.gy, K, M, 2 * a.ld_gy)) != SDQ_OK) return st;
   sdq::Params p;
-  p.giq = static_cast<int8_t*>(giq);
-  p.gis = gis;
-  p.yqt = static_cast<int8_t*>(yqt);
-  p.yst = yst;
+  p.giq = static_cast<int8_t*>(a.giq);
+  p.gis = a.gis;
+  p.yqt = static_cast<int8_t*>(a.yqt);
+  p.yst = a.yst;
   p.M = M;
   p.K = static_cast<int32_t>(K);
   p.Kg = static_cast<int32_t>(K / sdq::kG);
   p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
   p.gis_cols = static_cast<int32_t>(2 * K / group_size);
-  p.ys_groups = static_cast<int32_t>((M + group_size - 1) / group_size);
+  p.ld_giq = static_cast<int32_t>(a.ld_giq);
+  p.ld_gis = static_cast<int32_t>(a.ld_gis);
+  p.ld_yqt = a.ld_yqt;
+  p.ld_yst = a.ld_yst;
   p.num_tiles = p.Mg * p.Kg;
-  p.yqt_vec16 = (M % 16 == 0) ? 1 : 0;
+  p.yqt_vec16 = (a.ld_yqt % 16 == 0) ? 1 : 0;
   p.wait_limit_ns = limit_ns ? limit_ns : wait_limit_ns();
   p.withhold_first_load = withhold;
   const int grid = std::min(p.num_tiles, d->sms);
@@ -179,7 +217,7 @@ int launch(const void* x, const void* gy, void* giq, void* gis, void* yqt, void*
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format), mx, mg, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format), mgate, mup, mdy, p);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -235,13 +273,16 @@ const char* sdq_status_string(int status) {
     case SDQ_ERR_WORKSPACE: return "SDQ_ERR_WORKSPACE: workspace too small or misaligned";
     case SDQ_ERR_TOO_LARGE: return "SDQ_ERR_TOO_LARGE: K exceeds what fits in the fixed scratch of sdq_fuse_host_noalloc (SDQ_NOALLOC_MAX_K)";
     case SDQ_ERR_FORMAT: return "SDQ_ERR_FORMAT: unknown bits in the output format";
+    case SDQ_ERR_STRIDE: return "SDQ_ERR_STRIDE: a leading dimension is smaller than its row or above SDQ_MAX_LD";
     default: return "SDQ_ERR_UNKNOWN";
   }
 }
 
-int sdq_validate_format(const void* x, const void* grad_y, const void* grad_input_q,
-                        const void* grad_input_s, const void* y_q_t, const void* y_s_t, int64_t M,
-                        int64_t K, int32_t group_size, uint32_t format) {
+int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                         const void* grad_y, int64_t ld_grad_y, const void* grad_input_q,
+                         int64_t ld_grad_input_q, const void* grad_input_s, int64_t ld_grad_input_s,
+                         const void* y_q_t, int64_t ld_y_q_t, const void* y_s_t, int64_t ld_y_s_t,
+                         int64_t M, int64_t K, int32_t group_size, uint32_t format) {
   if (format & ~static_cast<uint32_t>(SDQ_FMT_E4M3 | SDQ_FMT_E8M0 | SDQ_FMT_YS_MG_K))
     return SDQ_ERR_FORMAT;
   if (!group_size_supported(group_size)) return SDQ_ERR_GROUP;
@@ -250,12 +291,33 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
   const int64_t tiles = ((M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE) * (K / SDQ_GROUP_SIZE);
   if (tiles > INT32_MAX) return SDQ_ERR_SHAPE;
   if (M == 0) return SDQ_OK;
-  if (!x || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t) return SDQ_ERR_NULL;
-  const uintptr_t a16 = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(grad_y) |
-                        reinterpret_cast<uintptr_t>(grad_input_q) | reinterpret_cast<uintptr_t>(y_q_t);
+  if (!gate || !up || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t)
+    return SDQ_ERR_NULL;
+  const int64_t groups_m = (M + group_size - 1) / group_size;
+  const int64_t need_yst = (format & SDQ_FMT_YS_MG_K) ? K : groups_m;
+  const int64_t lds[7] = {ld_gate, ld_up, ld_grad_y, ld_grad_input_q, ld_grad_input_s, ld_y_q_t, ld_y_s_t};
+  const int64_t need[7] = {K, K, K, 2 * K, 2 * K / group_size, M, need_yst};
+  for (int k = 0; k < 7; ++k)
+    if (lds[k] < need[k] || lds[k] > SDQ_MAX_LD) return SDQ_ERR_STRIDE;
+  if (ld_grad_input_q > SDQ_MAX_LD_ROWS || ld_grad_input_s > SDQ_MAX_LD_ROWS) return SDQ_ERR_STRIDE;
+  const uintptr_t a16 = reinterpret_cast<uintptr_t>(gate) | reinterpret_cast<uintptr_t>(up) |
+                        reinterpret_cast<uintptr_t>(grad_y) | reinterpret_cast<uintptr_t>(grad_input_q) |
+                        reinterpret_cast<uintptr_t>(y_q_t);
   const uintptr_t a4 = reinterpret_cast<uintptr_t>(grad_input_s) | reinterpret_cast<uintptr_t>(y_s_t);
   if ((a16 & 15u) || (!(format & SDQ_FMT_E8M0) && (a4 & 3u))) return SDQ_ERR_ALIGN;
+  // rows of the bf16 inputs start on 16 bytes (tensor-map strides), rows of
+  // grad_input_q on 16 bytes (vector stores)
+  if ((ld_gate | ld_up | ld_grad_y) & 7 || ld_grad_input_q & 15) return SDQ_ERR_ALIGN;
   return SDQ_OK;
+}
+
+int sdq_validate_format(const void* x, const void* grad_y, const void* grad_input_q,
+                        const void* grad_input_s, const void* y_q_t, const void* y_s_t, int64_t M,
+                        int64_t K, int32_t group_size, uint32_t format) {
+  const Arrays a = packed(x, grad_y, const_cast<void*>(grad_input_q), const_cast<void*>(grad_input_s),
+                          const_cast<void*>(y_q_t), const_cast<void*>(y_s_t), M, K, group_size, format);
+  return sdq_validate_strided(a.gate, a.ld_gate, a.up, a.ld_up, a.gy, a.ld_gy, a.giq, a.ld_giq, a.gis,
+                              a.ld_gis, a.yqt, a.ld_yqt, a.yst, a.ld_yst, M, K, group_size, format);
 }
 
 int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
@@ -270,8 +332,22 @@ int sdq_fuse_format(const void* x, const void* grad_y, void* grad_input_q, void*
   const int st = sdq_validate_format(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K,
                                      group_size, format);
   if (st != SDQ_OK || M == 0) return st;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, format,
-                static_cast<cudaStream_t>(stream));
+  return launch(packed(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, format),
+                M, K, group_size, format, static_cast<cudaStream_t>(stream));
+}
+
+int sdq_fuse_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                     const void* grad_y, int64_t ld_grad_y, void* grad_input_q,
+                     int64_t ld_grad_input_q, void* grad_input_s, int64_t ld_grad_input_s,
+                     void* y_q_t, int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t, int64_t M,
+                     int64_t K, int32_t group_size, uint32_t format, void* stream) {
+  const int st = sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
+                                      ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t,
+                                      y_s_t, ld_y_s_t, M, K, group_size, format);
+  if (st != SDQ_OK || M == 0) return st;
+  const Arrays a = {gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q, ld_grad_input_q,
+                    grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t};
+  return launch(a, M, K, group_size, format, static_cast<cudaStream_t>(stream));
 }
 
 int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q, float* grad_input_s,
@@ -348,8 +424,9 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
     SDQ_CHECK(cudaEventRecord(d->in_ready[b], d->h2d));
     // kernel on the caller's stream
     SDQ_CHECK(cudaStreamWaitEvent(cs, d->in_ready[b], 0));
-    st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt, base + L.yst, mc,
-                K, SDQ_GROUP_SIZE, 0, cs);
+    st = launch(packed(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt, base + L.yst,
+                       mc, K, SDQ_GROUP_SIZE, 0),
+                mc, K, SDQ_GROUP_SIZE, 0, cs);
     if (st != SDQ_OK) return st;
     SDQ_CHECK(cudaEventRecord(d->out_ready[b], cs));
     // device -> host
@@ -440,8 +517,9 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
     if ((e = cudaMemcpyAsync(base + L.gy, gh + m0 * 2 * K, size_t(mc) * 2 * K,
                              cudaMemcpyHostToDevice, cs)) != cudaSuccess)
       return cuda_fail(e);
-    const int st = launch(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt,
-                          base + L.yst, mc, K, SDQ_GROUP_SIZE, 0, cs);
+    const int st = launch(packed(base + L.x, base + L.gy, base + L.giq, base + L.gis, base + L.yqt,
+                                 base + L.yst, mc, K, SDQ_GROUP_SIZE, 0),
+                          mc, K, SDQ_GROUP_SIZE, 0, cs);
     if (st != SDQ_OK) return st;
     if ((e = cudaMemcpyAsync(grad_input_q + m0 * 2 * K, base + L.giq, size_t(mc) * 2 * K,
                              cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
@@ -466,8 +544,9 @@ int sdq_fuse_test_stall(const void* x, const void* grad_y, int8_t* grad_input_q,
   const int st = sdq_validate(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size);
   if (st != SDQ_OK || M == 0) return st;
   if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000) return SDQ_ERR_SHAPE;
-  return launch(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, 0,
-                static_cast<cudaStream_t>(stream), static_cast<uint64_t>(wait_limit_ns), 1);
+  return launch(packed(x, grad_y, grad_input_q, grad_input_s, y_q_t, y_s_t, M, K, group_size, 0), M,
+                K, group_size, 0, static_cast<cudaStream_t>(stream), static_cast<uint64_t>(wait_limit_ns),
+                1);
 }
 
 int sdq_device_status(void* stream) {

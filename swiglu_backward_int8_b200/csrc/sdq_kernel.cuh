@@ -85,11 +85,14 @@ struct Params {
   int64_t M;
   int32_t K;
   int32_t Kg;        // 128-channel tiles per row
-  int32_t gis_cols;  // 2K / group size: columns of grad_input_s
-  int32_t ys_groups; // ceil(M / group size): token groups of y_s_t
+  int32_t gis_cols;  // 2K / group size: columns of grad_input_s (d_up groups from gis_cols/2)
+  int64_t ld_yqt;    // elements from one row of each output to the next
+  int64_t ld_yst;
+  int32_t ld_giq;    // (at most 2^24: a tile's row offsets stay 32-bit products)
+  int32_t ld_gis;
   int32_t Mg;
   int32_t num_tiles;
-  int32_t yqt_vec16;  // M % 16 == 0: y_q_t rows take 16-byte stores
+  int32_t yqt_vec16;  // ld_yqt % 16 == 0: y_q_t rows take 16-byte stores
   int32_t withhold_first_load;  // test hook: leave load 0 unissued so its wait runs out
   uint64_t wait_limit_ns;
 };
@@ -133,10 +136,12 @@ __device__ __forceinline__ void tile_ij(int t, int Mg, int Kg, int& i, int& j) {
 }
 
 // Load n of this CTA: stage n % 2 of its (n / 2)-th tile, into slot n % STAGES.
+// The three input tensor maps (gate, up, grad_y: [M, K] bf16 each, with their
+// own row strides; gate and up may be the two halves of one x = [gate | up]).
 template <int STAGES>
-__device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* mx,
-                                           const CUtensorMap* mg, const Params& p, uint32_t n,
-                                           uint64_t pol) {
+__device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* mgate,
+                                           const CUtensorMap* mup, const CUtensorMap* mdy,
+                                           const Params& p, uint32_t n, uint64_t pol) {
   const int t = blockIdx.x + static_cast<int>(n / kStagesPerTile) * gridDim.x;
   int i, j;
   tile_ij(t, p.Mg, p.Kg, i, j);
@@ -145,9 +150,9 @@ __device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* m
   const uint32_t fb = smem_u32(&s.full[slot]);
   mbar_arrive_expect_tx(fb, kStageBytes);
   const uint32_t dst = smem_u32(s.ring[slot]);
-  tma_load_2d(dst, mx, fb, j * kG, r, pol);                          // gate
-  tma_load_2d(dst + kBoxBytes, mx, fb, p.K + j * kG, r, pol);        // up
-  tma_load_2d(dst + 2 * kBoxBytes, mg, fb, j * kG, r, pol);          // grad_y
+  tma_load_2d(dst, mgate, fb, j * kG, r, pol);
+  tma_load_2d(dst + kBoxBytes, mup, fb, j * kG, r, pol);
+  tma_load_2d(dst + 2 * kBoxBytes, mdy, fb, j * kG, r, pol);
 }
 
 // bf16 pair -> two floats (exact).
@@ -376,7 +381,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   const int tg = kc / kTpg;        // token group within the tile
   if (gk < 2 && tg * kGS < valid) {
     const int64_t grp = int64_t(i) * (kG / kGS) + tg;
-    store_scale<kE8M0>(p.yst, kYsMgK ? grp * p.K + ch + gk : int64_t(ch + gk) * p.ys_groups + grp,
+    store_scale<kE8M0>(p.yst, kYsMgK ? grp * p.ld_yst + ch + gk : int64_t(ch + gk) * p.ld_yst + grp,
                        gk ? s_hi : s_lo);
   }
   uint4 lo, hi;
@@ -390,15 +395,16 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   const int tok = 16 * kc;
   if (tok < valid) {
     const int nb = min(16, valid - tok);
-    int8_t* dst = p.yqt + int64_t(ch) * p.M + row0 + tok;
+    int8_t* dst = p.yqt + int64_t(ch) * p.ld_yqt + row0 + tok;
     store_codes(dst, lo, nb, p.yqt_vec16 != 0);
-    store_codes(dst + p.M, hi, nb, p.yqt_vec16 != 0);
+    store_codes(dst + p.ld_yqt, hi, nb, p.yqt_vec16 != 0);
   }
 }
 
 template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK>
 __global__ void __launch_bounds__(kThreads, 1)
-    fuse_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy,
+    fuse_kernel(const __grid_constant__ CUtensorMap map_gate, const __grid_constant__ CUtensorMap map_up,
+                const __grid_constant__ CUtensorMap map_gy,
                 const Params p) {
   constexpr unsigned kFull = 0xffffffffu;
   extern __shared__ uint8_t smem_raw[];
@@ -423,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid < 128) s.scale_tab[tid] = scale_table_entry<kE4M3, kE8M0>(tid);
   if (tid == 0) {
-    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_gate);
+    prefetch_tensormap(&map_up);
     prefetch_tensormap(&map_gy);
     for (int st = 0; st < STAGES; ++st) {
       mbar_init(smem_u32(&s.full[st]), 1);
@@ -439,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t first = total < STAGES ? total : STAGES;
     s.issued = static_cast<int>(first);
     for (uint32_t n = 0; n < first; ++n)
-      if (n != 0 || !p.withhold_first_load) issue_load(s, &map_x, &map_gy, p, n, pol);
+      if (n != 0 || !p.withhold_first_load) issue_load(s, &map_gate, &map_up, &map_gy, p, n, pol);
   }
   grid_dependency_wait();   // every thread: global memory only after the previous grid is done
   grid_launch_dependents();
@@ -471,9 +478,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int yb = k % kYBuf;   // y buffer of this tile; tile t completes phase t / kYBuf of its barriers
     uint8_t* yt = s.ytile[yb];
     // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
-    int8_t* giq_t = p.giq + row0 * (2 * int64_t(K)) + j * kG;
+    int8_t* giq_t = p.giq + row0 * p.ld_giq + j * kG;
     // scale index of (row0, the tile's first d_gate group)
-    const int64_t gis_t = row0 * p.gis_cols + j * (kG / kGS);
+    const int64_t gis_t = row0 * p.ld_gis + j * (kG / kGS);
 
     // ================= row pass over the tile's two stages
 #pragma unroll
@@ -509,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t nn = n + STAGES;
           if (nn < total) {
             atomicMax(&s.issued, static_cast<int>(nn + 1));
-            issue_load(s, &map_x, &map_gy, p, nn, pol);
+            issue_load(s, &map_gate, &map_up, &map_gy, p, nn, pol);
           }
         }
       }
@@ -556,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kLpg = kGS / 16;   // lanes per channel group
         const int gl = cq & (kLpg - 1);
         if (gl < 2 && rbase + rr < valid)
-          store_scale<kE8M0>(p.gis, gis_t + int64_t(rbase + rr) * p.gis_cols + cq / kLpg +
+          store_scale<kE8M0>(p.gis, gis_t + (rbase + rr) * p.ld_gis + cq / kLpg +
                                         gl * (p.gis_cols >> 1),
                              gl ? su : sg);
       }
@@ -572,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           og = quant16<kE4M3, false>(dgp, ig);
           ou = quant16<kE4M3, false>(dup, iu);
         }
-        int8_t* dst = giq_t + r * (2 * K);
+        int8_t* dst = giq_t + r * p.ld_giq;
         st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
         st_cs_v2(dst + cb * 8, make_uint2(og.z, og.w));
         st_cs_v2(dst + K + ca * 8, make_uint2(ou.x, ou.y));

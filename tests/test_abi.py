@@ -159,3 +159,56 @@ def test_format_names_shapes_and_dtypes():
         sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, q, s, yq, ys.T.contiguous(), y_scale_layout="mg_k")
     with pytest.raises(ValueError):     # E4M3 codes with INT8 asked for
         sdq.silu_dot_fwd_bwd_quant_fuse(x, gy, q, s, yq, ys, codes="int8", y_scale_layout="mg_k")
+
+
+def _strided_args(**kw):
+    M, K = 256, 256
+    a = dict(gate=A, ld_gate=2 * K, up=A + 2 * K, ld_up=2 * K, grad_y=A, ld_grad_y=K,
+             grad_input_q=A, ld_grad_input_q=2 * K, grad_input_s=A, ld_grad_input_s=4,
+             y_q_t=A, ld_y_q_t=M, y_s_t=A, ld_y_s_t=2, M=M, K=K, group_size=128, format=0)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0),
+    (dict(ld_gate=1024, ld_up=520, ld_grad_y=264, ld_grad_input_q=528, ld_grad_input_s=7,
+          ld_y_q_t=259, ld_y_s_t=9), 0),                  # padded rows; y_q_t ld not a multiple of 16
+    (dict(up=A + (1 << 20)), 0),                         # gate and up apart
+    (dict(ld_gate=255), 10),                             # shorter than a row
+    (dict(ld_grad_input_s=3), 10),
+    (dict(ld_y_q_t=255), 10),
+    (dict(ld_y_s_t=1), 10),
+    (dict(format=4, ld_y_s_t=255), 10),                  # [Mg, K] layout needs ld >= K
+    (dict(format=4, ld_y_s_t=256), 0),
+    (dict(ld_gate=1 << 37), 10),                         # above SDQ_MAX_LD
+    (dict(ld_grad_input_q=(1 << 24) + 16), 10),          # above SDQ_MAX_LD_ROWS
+    (dict(ld_grad_input_s=(1 << 24) + 1), 10),
+    (dict(ld_up=516), 4),                                # bf16 rows must start on 16 bytes
+    (dict(ld_grad_input_q=520), 4),                      # grad_input_q rows on 16 bytes
+    (dict(up=A + 8), 4),
+    (dict(group_size=64, ld_grad_input_s=8, ld_y_s_t=4), 0),
+    (dict(group_size=64, ld_grad_input_s=7), 10),
+    (dict(M=0, gate=0, up=0), 0),
+    (dict(up=0), 1),
+])
+def test_validate_strided_statuses(kw, status):
+    import swiglu_backward_int8_b200 as sdq
+    a = _strided_args(**kw)
+    assert sdq.sdq_validate_strided(*a.values()) == status
+
+
+def test_wrapper_takes_row_strides_and_refuses_other_layouts():
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    from swiglu_backward_int8_b200 import _rows
+    wide = torch.zeros(8, 600, dtype=torch.bfloat16)
+    assert _rows("x", wide, (8, 600), (torch.bfloat16,), False, None) == 600
+    with pytest.raises(ValueError):          # transposed: rows are not unit-stride
+        _rows("x", torch.zeros(512, 8, dtype=torch.bfloat16).t(), (8, 512), (torch.bfloat16,), True,
+              torch.device("cpu"))
+    with pytest.raises(ValueError):          # expanded: rows overlap
+        _rows("x", torch.zeros(1, 512, dtype=torch.bfloat16).expand(8, 512), (8, 512),
+              (torch.bfloat16,), True, torch.device("cpu"))
+    with pytest.raises(ValueError):          # the host entry points need contiguous tensors
+        _rows("x", wide[:, :512], (8, 512), (torch.bfloat16,), False, torch.device("cpu"))
