@@ -73,6 +73,12 @@ def lib() -> ctypes.CDLL:
         L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.argtypes = [P, P, P, P, P, P, i64, i64, i64,
                                                              ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.restype = ctypes.c_int
+        L.oracle_fp16_rne.argtypes = [dbl]
+        L.oracle_fp16_rne.restype = ctypes.c_uint16
+        L.oracle_q8_1_block.argtypes = [P, P]
+        L.oracle_q8_1_block.restype = None
+        L.oracle_swiglu_q8_1_rows.argtypes = [P, P, P, P, P, i64, i64, ctypes.c_float]
+        L.oracle_swiglu_q8_1_rows.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -223,3 +229,43 @@ def silu_dot_fwd_bwd_quant_fuse_fmt(x: np.ndarray, grad_y: np.ndarray, group_siz
         raise ValueError(f"oracle rejected M={M} K={K} group_size={G} format "
                          f"({codes}, {scales}, {ys_layout})")
     return giq, gis, yqt, yst
+
+
+# ---- forward-side neighbour: SwiGLU forward + q8_1 rows ----------------------
+
+Q8_1_BLOCK_BYTES = 36
+
+
+def fp16_rne(v: float) -> int:
+    """Nearest IEEE binary16 bit pattern of a double, ties to even."""
+    return int(lib().oracle_fp16_rne(float(v)))
+
+
+def q8_1_block(h_bf16: np.ndarray) -> np.ndarray:
+    """One 36-byte q8_1 block (fp16 d, fp16 sum, 32 int8) of 32 bf16 values."""
+    h = np.ascontiguousarray(h_bf16, dtype=np.uint16)
+    assert h.size == 32
+    out = np.zeros(Q8_1_BLOCK_BYTES, np.uint8)
+    lib().oracle_q8_1_block(_ptr(h), _ptr(out))
+    return out
+
+
+def swiglu_q8_1_rows(gate: np.ndarray, up: np.ndarray, w=None, limit: float = 0.0):
+    """The forward op on uint16 (bf16 bit) arrays [rows, inter]; w float32 [rows]
+    or None.  Returns (h [rows, inter] uint16 bf16 bits, q8 [rows, inter/32, 36] uint8)."""
+    g = np.ascontiguousarray(gate, dtype=np.uint16)
+    u = np.ascontiguousarray(up, dtype=np.uint16)
+    rows, inter = g.shape
+    assert u.shape == g.shape
+    h = np.zeros((rows, inter), np.uint16)
+    q8 = np.zeros((rows, inter // 32, Q8_1_BLOCK_BYTES), np.uint8)
+    wp = None
+    if w is not None:
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        assert w.shape == (rows,)
+        wp = _ptr(w)
+    rc = lib().oracle_swiglu_q8_1_rows(_ptr(g), _ptr(u), wp, _ptr(h), _ptr(q8), rows, inter,
+                                       float(limit))
+    if rc != 0:
+        raise ValueError(f"oracle rejected rows={rows} inter={inter}")
+    return h, q8

@@ -57,6 +57,19 @@
 //   * In every format an all-zero group has scale 1 and each code is that of
 //     v / 1: zero, with v's sign in E4M3 (0x80 for -0.0).
 //   * y_s_t [Mg, K]: token group i, channel k at i * K + k.
+// The forward-side neighbour (the q8_1 activation path on the page whose
+// launcher is kquant_swiglu_q8_1_rows: "h = bf16(swiglu(gate, up) * w[row]),
+// then the q8_1 blocks of those bf16 rows"; a block_q8_1 is "32 int8 + half2
+// (d, sum)", 36 bytes).  Readings where that page is silent: swiglu(g, u) =
+// silu(g) * u as in the backward op, with `limit` > 0 clamping gate to at
+// most limit and up to [-limit, limit] first (limit <= 0 or NaN: no clamp);
+// h in fp64 rounded once to bf16; per block of 32 consecutive h values of a
+// row, d32 = fl32(amax / 127), q = round-half-even(fl32(h / d32)) in
+// [-127, 127], stored d = fp16(d32) and sum = fp16(d32 * sum(q)) (the exact
+// product rounded once: the sum of the block's dequantized values), both
+// nearest-even; an all-zero block has d = sum = 0 and q = 0; the block is
+// half2 (d, sum) first, then the 32 codes.  Pins: tests/test_oracle_fwd.py.
+//
 // Pins (tests/test_oracle_formats.py): oracle_e4m3_rne against torch's
 // float8_e4m3fn conversion inside the finite range and against brute force
 // over all 127 finite magnitudes with exact rationals; oracle_e8m0_ceil
@@ -328,6 +341,83 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
       oracle_quant_group_fmt(&y[t0 * K + k], n, K, &y_q_t[k * M + t0], 1, yst + si * sb, codes,
                              scales);
     }
+  }
+  return 0;
+}
+
+// ---- forward-side neighbour: SwiGLU forward + q8_1 rows -----------------------
+
+// Nearest IEEE binary16 of a double, ties to even, subnormals kept, overflow
+// to infinity; returns the bit pattern.
+uint16_t oracle_fp16_rne(double v) {
+  if (std::isnan(v)) return 0x7E00;
+  const uint16_t sign = std::signbit(v) ? 0x8000 : 0x0000;
+  const double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e = std::ilogb(a);
+  if (e < -14) e = -14;                      // below the normal range the spacing stays 2^-24
+  const double ulp = std::ldexp(1.0, e - 10);
+  const double r = std::nearbyint(a / ulp) * ulp;
+  if (r >= 65520.0) return sign | 0x7C00;   // 65504 + half its spacing rounds up to infinity
+  if (r < std::ldexp(1.0, -14)) return sign | static_cast<uint16_t>(r / std::ldexp(1.0, -24));
+  const int re = std::ilogb(r);
+  const int mant = static_cast<int>(r / std::ldexp(1.0, re - 10)) - 1024;
+  return sign | static_cast<uint16_t>(((re + 15) << 10) | mant);
+}
+
+// One row's h values (bf16 bits) for gate/up rows g, u of length n and row
+// weight w (already 1 when there is none).
+void oracle_swiglu_row(const uint16_t* g, const uint16_t* u, double w, int64_t n, double limit,
+                       uint16_t* h) {
+  for (int64_t k = 0; k < n; ++k) {
+    double gv = bf16_to_float(g[k]);
+    double uv = bf16_to_float(u[k]);
+    if (limit > 0.0) {   // false for NaN: no clamp
+      gv = gv < limit ? gv : limit;
+      uv = uv < -limit ? -limit : (uv > limit ? limit : uv);
+    }
+    h[k] = oracle_bf16_rne(oracle_silu(gv) * uv * w);
+  }
+}
+
+// One q8_1 block (36 bytes: fp16 d, fp16 sum, 32 int8) from 32 bf16 values.
+void oracle_q8_1_block(const uint16_t* h, uint8_t* out) {
+  float amax = 0.0f;
+  for (int i = 0; i < 32; ++i) {
+    const float a = std::fabs(bf16_to_float(h[i]));
+    if (a > amax) amax = a;
+  }
+  int8_t q[32] = {0};
+  uint16_t d16 = 0, s16 = 0;
+  if (amax != 0.0f) {
+    const float d = amax / 127.0f;
+    long qsum = 0;
+    for (int i = 0; i < 32; ++i) {
+      float r = std::nearbyint(bf16_to_float(h[i]) / d);
+      if (r > 127.0f) r = 127.0f;
+      if (r < -127.0f) r = -127.0f;
+      q[i] = static_cast<int8_t>(r);
+      qsum += q[i];
+    }
+    d16 = oracle_fp16_rne(d);
+    s16 = oracle_fp16_rne(static_cast<double>(d) * static_cast<double>(qsum));  // exact product
+  }
+  std::memcpy(out, &d16, 2);
+  std::memcpy(out + 2, &s16, 2);
+  std::memcpy(out + 4, q, 32);
+}
+
+// The forward op: gate, up [rows, inter] bf16; w [rows] fp32 or NULL;
+// h [rows, inter] bf16; q8 [rows, inter/32] blocks of 36 bytes.  Returns 0,
+// or -1 when inter is not a positive multiple of 32 or rows < 0.
+int oracle_swiglu_q8_1_rows(const uint16_t* gate, const uint16_t* up, const float* w,
+                            uint16_t* h, uint8_t* q8, int64_t rows, int64_t inter, float limit) {
+  if (rows < 0 || inter < 32 || inter % 32 != 0) return -1;
+  for (int64_t m = 0; m < rows; ++m) {
+    const double wm = w ? static_cast<double>(w[m]) : 1.0;
+    oracle_swiglu_row(&gate[m * inter], &up[m * inter], wm, inter, limit, &h[m * inter]);
+    for (int64_t b = 0; b < inter / 32; ++b)
+      oracle_q8_1_block(&h[m * inter + b * 32], &q8[(m * (inter / 32) + b) * 36]);
   }
   return 0;
 }

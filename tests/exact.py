@@ -144,3 +144,24 @@ def pow2_ceil_exponent(v: Fraction) -> int:
     """Smallest k with 2^k >= v (v > 0)."""
     k = _floor_log2(v)
     return k if Fraction(2) ** k == v else k + 1
+
+
+def fp16_nearest(v: Fraction) -> int:
+    """IEEE binary16 bit pattern nearest to an exact rational, by comparing the
+    exact distance to every finite half value near a start point (ties to the
+    even pattern; at or beyond 65520 infinity)."""
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    if a >= 65520:
+        return sign | 0x7C00
+    with np.errstate(over="ignore"):
+        start = int(np.array([float(a)], np.float64).astype(np.float16).view(np.uint16)[0])
+    start = min(start, 0x7BFF)
+    best = None
+    for bits in range(max(0, start - 4), min(0x7BFF, start + 4) + 1):   # a start point +- 4 patterns
+        f, m = bits >> 10, bits & 0x3FF
+        val = Fraction(m, 2 ** 24) if f == 0 else (1 + Fraction(m, 1024)) * Fraction(2) ** (f - 15)
+        key = (abs(val - a), bits & 1)
+        if best is None or key < best[0]:
+            best = (key, bits)
+    return sign | best[1]

@@ -54,9 +54,25 @@ MUTATIONS = [
      "test_whole_op_fmt_ys_layouts_transpose", "formats"),
     ("oracle_quant_group_fmt(&y[t0 * K + k], n, K,", "oracle_quant_group_fmt(&y[t0 * K + k], n, 1,",
      "test_whole_op_fmt_groups_relate_to_stage1", "formats"),
+    # forward-side neighbour (pins in test_oracle_fwd.py)
+    ("if (e < -14) e = -14;", "", "test_fp16_rne_against_numpy_float16_conversion", "fwd"),
+    ("const int mant = static_cast<int>(r / std::ldexp(1.0, re - 10)) - 1024;",
+     "const int mant = static_cast<int>(r / std::ldexp(1.0, re - 10)) - 1023;",
+     "test_fp16_rne_against_numpy_float16_conversion", "fwd"),
+    ("gv = gv < limit ? gv : limit;", "gv = gv < -limit ? -limit : (gv > limit ? limit : gv);",
+     "test_swiglu_rows_limit_clamps_gate_above_and_up_both_ways", "fwd"),
+    ("h[k] = oracle_bf16_rne(oracle_silu(gv) * uv * w);", "h[k] = oracle_bf16_rne(oracle_silu(gv) * uv);",
+     "test_swiglu_rows_closed_form_without_clamp", "fwd"),
+    ("s16 = oracle_fp16_rne(static_cast<double>(d) * static_cast<double>(qsum));  // exact product",
+     "s16 = oracle_fp16_rne(static_cast<double>(qsum));", "test_q8_1_block_against_its_definition", "fwd"),
+    ("&q8[(m * (inter / 32) + b) * 36]", "&q8[(b * rows + m) * 36]",
+     "test_swiglu_rows_blocks_are_the_rows_32_value_blocks", "fwd"),
+    ("if (limit > 0.0) {   // false for NaN: no clamp", "if (limit != 0.0) {",
+     "test_swiglu_rows_closed_form_without_clamp", "fwd"),
 ]
 
-PIN_FILES = {"pins": "test_oracle_pins.py", "formats": "test_oracle_formats.py"}
+PIN_FILES = {"pins": "test_oracle_pins.py", "formats": "test_oracle_formats.py",
+             "fwd": "test_oracle_fwd.py"}
 
 
 def _run_mutant(tmp_dir, idx, old, new, pin, pins="pins"):
