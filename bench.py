@@ -48,6 +48,9 @@ import workloads as W  # noqa: E402
 DEFAULT_WORKLOAD = W.WORKLOADS[1].name
 METRIC = "µs/call and achieved HBM GB/s (fraction of B200 roofline) per (M,K)"
 FALLBACK_HBM_GBS = 6650.0
+FWD_SOURCES = ["swiglu_backward_int8_b200/csrc/fwd_kernel.cuh",
+               "swiglu_backward_int8_b200/csrc/fwd_api.cu",
+               "swiglu_backward_int8_b200/csrc/sdq_ptx.cuh"]
 KERNEL_SOURCES = ["swiglu_backward_int8_b200/csrc/sdq_kernel.cuh",
                   "swiglu_backward_int8_b200/csrc/sdq_ptx.cuh",
                   "swiglu_backward_int8_b200/csrc/sdq_api.cu"]
@@ -70,6 +73,10 @@ def parse_args():
     ap.add_argument("--scales", choices=["fp32", "e8m0"], default="fp32",
                     help="scale format of the timed calls (the page's: fp32)")
     ap.add_argument("--y-scale-layout", choices=["k_mg", "mg_k"], default="k_mg")
+    ap.add_argument("--op", choices=["fuse", "swiglu_q8_1"], default="fuse",
+                    help="fuse: the backward op (the headline); swiglu_q8_1: the forward-side "
+                         "SwiGLU + q8_1 rows on the workload's gate and up (rows = M, inter = K)")
+    ap.add_argument("--limit", type=float, default=0.0, help="swiglu_q8_1: the clamp (0: none)")
     ap.add_argument("--all-formats", action="store_true",
                     help="also time every output format on the workload and add a per_format list")
     a = ap.parse_args()
@@ -86,9 +93,9 @@ def pick_workload(name: str) -> W.Workload:
     return W.BY_NAME[name]
 
 
-def kernel_sha() -> str:
+def kernel_sha(sources=None) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (sources or KERNEL_SOURCES):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -467,10 +474,126 @@ def run_sdq(args):
     return 0
 
 
+FWD_METRIC = "µs/call and achieved HBM GB/s (fraction of B200 roofline): SwiGLU forward + q8_1 rows"
+
+
+def fwd_bytes(rows: int, inter: int, with_w: bool = True) -> int:
+    """Algorithmic bytes of the forward op: read gate and up (4 B per element)
+    and the row weights, write h (2 B) and the q8_1 blocks (36 B per 32)."""
+    return rows * inter * 6 + rows * (inter // 32) * 36 + (4 * rows if with_w else 0)
+
+
+def run_fwd(args):
+    """The forward-side neighbour on one GPU: device-timed like the backward
+    op (CUDA-graph replay, buffers rotating through >= 3x L2)."""
+    import torch
+    world, rank, local = dist_setup(args)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import swiglu_backward_int8_b200 as sdq  # fails loudly if the CUDA library is missing
+    from swiglu_backward_int8_b200 import parallel
+    parallel.init_from_env("nccl", timeout_s=120.0, device=device)
+    w = pick_workload(args.workload)
+    rows, inter = w.M, w.K
+    g_np, u_np, wt_np = W.fwd_inputs(W.Workload(w.name, w.M, w.K, w.sigma_x, w.sigma_grad_y,
+                                                w.seed + 1000 * rank, w.group_size, w.outlier_frac,
+                                                w.outlier_mult, w.zero_group_every))
+    peak, peak_kind = measured_peaks()
+    nbytes = fwd_bytes(rows, inter)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, -(-3 * l2 // nbytes))
+    x0 = _to_device_bf16(np.concatenate([g_np, u_np], axis=1), device)
+    wt0 = torch.from_numpy(wt_np).to(device)
+    sets = []
+    for k in range(nsets):
+        xs = x0 if k == 0 else x0.clone()
+        sets.append((xs, wt0 if k == 0 else wt0.clone(),
+                     torch.empty((rows, inter), dtype=torch.bfloat16, device=device),
+                     torch.empty((rows, inter // 32, 36), dtype=torch.uint8, device=device)))
+
+    def call(k):
+        xs, wt, h, q8 = sets[k % nsets]
+        sdq.swiglu_q8_1(xs[:, :inter], xs[:, inter:], wt, args.limit, h, q8)
+
+    for k in range(args.warmup):
+        call(k)
+    torch.cuda.synchronize(device)
+    graphs, done = [], 0
+    while done < args.steps:
+        n = min(1000, args.steps - done)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+            for k in range(n):
+                call(args.warmup + done + k)
+        graphs.append(g)
+        done += n
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream(device)
+    parallel.barrier(device)
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    ev0.record(stream)
+    for g in graphs:
+        g.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    clocks = sampler.summary(t0, t1)
+    sampler.stop()
+    ms = parallel.max_over_ranks(ev0.elapsed_time(ev1), device)
+    per_ms = ms / args.steps
+    achieved = nbytes / (per_ms * 1e-3) / 1e9
+    value = parallel.aggregate_gbs(nbytes * args.steps, world, ms)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        r = min(rows, 512)
+        gs, us, ws = (np.ascontiguousarray(g_np[:r]), np.ascontiguousarray(u_np[:r]), wt_np[:r])
+        oracle.swiglu_q8_1_rows(gs[:1], us[:1], ws[:1])
+        reps, c0 = 0, time.perf_counter()
+        while time.perf_counter() - c0 < 10.0:
+            oracle.swiglu_q8_1_rows(gs, us, ws, args.limit)
+            reps += 1
+        el = time.perf_counter() - c0
+        cpu = {"value": fwd_bytes(r, inter) * reps / el / 1e9, "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "sample": f"first {r} of {rows} rows x inter={inter}, {reps} "
+                                           f"repetitions in {el:.1f} s (single-threaded C++ oracle, fp64)"}
+    if rank == 0:
+        print(json.dumps({
+            "metric": FWD_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_ms, "us_per_call": per_ms * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name + "_swiglu_q8_1", "rows": rows, "inter": inter,
+                       "limit": args.limit, "row_weights": "uniform (0, 1]",
+                       "io": "bf16 gate, up, fp32 w in; bf16 h + q8_1 blocks out",
+                       "parallelism": f"replicas x{world} (no exchange)",
+                       "l2": f"inputs+outputs rotate over {nsets} buffer sets (>= 3x L2)",
+                       "timing": "K calls replayed from CUDA graphs, CUDA events"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes_per_launch": nbytes, "kernel": "sdq::fwd::swiglu_q8_1_kernel"},
+            "cpu_baseline": cpu,
+            "e2e": {"unavailable": "the forward op has a device entry point only"},
+            "gpu_launches": args.steps, "clocks": clocks, "kernel_sources_sha": kernel_sha(FWD_SOURCES),
+        }), flush=True)
+    del graphs
+    import torch.distributed as tdist
+    if tdist.is_initialized():
+        parallel.barrier(device)
+        tdist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "swiglu_q8_1":
+        return run_fwd(args)
     return run_sdq(args)
 
 

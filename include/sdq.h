@@ -191,6 +191,41 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
                          int32_t group_size, uint32_t format);
 
 /*
+ * sdq_swiglu_q8_1 -- the forward-side neighbour of the backward op: the
+ * SwiGLU forward and the q8_1 row quantization of its output in one pass.
+ * Source: the launcher kquant_swiglu_q8_1_rows on the page with the K-quant
+ * kernels ("h[rows, inter] = bf16(swiglu(gate, up) * w[row]), then the q8_1
+ * blocks of those bf16 rows"; "block_q8_1: 32 int8 + half2 (d, sum)", 36
+ * bytes; inter a multiple of 32).  Definitions where that page is silent:
+ *   h[m, k] = bf16(silu(g) * u * w[m]), computed in fp32, rounded once to
+ *   bf16 (nearest even); with limit > 0, g = min(gate, limit) and
+ *   u = clamp(up, -limit, limit) first (limit <= 0 or NaN: no clamp);
+ *   per block of 32 consecutive h of a row: d32 = fl32(amax / 127),
+ *   q = round-half-even(h * (1/d32)) in [-127, 127], d = fp16(d32),
+ *   sum = fp16(d32 * sum(q)); an all-zero block is all zero; a block is
+ *   half2 (d, sum) first (d in the low half), then the 32 codes.
+ *   gate, up   device, bf16 [rows, inter], 16-byte aligned, ld a multiple of 8
+ *   w          device, fp32 [rows] (a per-row weight, e.g. a router
+ *              weight), 4-byte aligned; NULL = 1
+ *   h          device, bf16 [rows, inter], 16-byte aligned, ld a multiple of 8
+ *              (written)
+ *   q8         device, [rows, inter/32] blocks of 36 bytes, contiguous,
+ *              4-byte aligned (written)
+ *   rows       0 <= rows <= SDQ_MAX_M (0: no-op); inter: a multiple of 32,
+ *              32 <= inter <= SDQ_MAX_K; ld_* in elements, >= inter
+ * One streaming kernel on `stream`; allocates nothing.  Errors as sdq_fuse
+ * (SDQ_ERR_SHAPE, SDQ_ERR_NULL, SDQ_ERR_STRIDE, SDQ_ERR_ALIGN, SDQ_ERR_CUDA).
+ */
+int sdq_swiglu_q8_1(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                    const float* w, void* h, int64_t ld_h, void* q8, int64_t rows,
+                    int64_t inter, float limit, void* stream);
+
+/* The argument checks of sdq_swiglu_q8_1 alone: no CUDA call, no launch. */
+int sdq_validate_swiglu_q8_1(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                             const float* w, const void* h, int64_t ld_h, const void* q8,
+                             int64_t rows, int64_t inter);
+
+/*
  * sdq_fuse_host -- the op on HOST buffers (same shapes and layouts as
  * sdq_fuse; page-locked host memory gives overlapped copies, pageable memory
  * works but copies synchronously).  The rows are processed in chunks through

@@ -24,11 +24,13 @@ import torch
 from ._lib import (FMT_E4M3, FMT_E8M0, FMT_YS_MG_K, LIB_PATH, SdqError, Status, last_cuda_error,
                    sdq_device_status, sdq_fuse, sdq_fuse_format, sdq_fuse_host,
                    sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_fuse_strided,
-                   sdq_validate, sdq_validate_format, sdq_validate_strided, status_string, version)
+                   sdq_swiglu_q8_1, sdq_validate, sdq_validate_format, sdq_validate_strided,
+                   sdq_validate_swiglu_q8_1, status_string, version)
 
 __all__ = [
     "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_split",
     "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs", "sdq_fuse_strided", "sdq_validate_strided",
+    "swiglu_q8_1", "sdq_swiglu_q8_1", "sdq_validate_swiglu_q8_1", "Q8_1_BLOCK_BYTES",
     "output_shapes", "output_format", "sdq_fuse", "sdq_fuse_format", "sdq_validate_format",
     "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
     "sdq_fuse_host_workspace_bytes", "sdq_validate",
@@ -214,6 +216,46 @@ def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
                       chunk_rows, stream)
         if synchronize:
             torch.cuda.current_stream(dev).synchronize()
+
+
+Q8_1_BLOCK_BYTES = 36
+
+
+def swiglu_q8_1(gate: torch.Tensor, up: torch.Tensor, w: Optional[torch.Tensor] = None,
+                limit: float = 0.0, h: Optional[torch.Tensor] = None,
+                q8: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The forward-side neighbour: h = bf16(silu(gate) * up * w[row]) (gate and
+    up clamped when limit > 0) and its q8_1 blocks, on the current CUDA stream.
+    gate, up: bf16 [rows, inter] (row-major, rows may be padded); w: fp32
+    [rows] or None.  Returns (h bf16 [rows, inter], q8 uint8 [rows, inter/32, 36]),
+    allocating whichever is not given."""
+    if gate.dim() != 2:
+        raise ValueError("gate must be 2-D")
+    rows, inter = gate.shape
+    if inter % 32 or inter < 32:
+        raise ValueError(f"inter={inter} must be a positive multiple of 32")
+    bf16 = (torch.bfloat16,)
+    ld_g = _rows("gate", gate, (rows, inter), bf16, True, gate.device)
+    ld_u = _rows("up", up, (rows, inter), bf16, True, gate.device)
+    if h is None:
+        h = torch.empty((rows, inter), dtype=torch.bfloat16, device=gate.device)
+    ld_h = _rows("h", h, (rows, inter), bf16, True, gate.device)
+    if q8 is None:
+        q8 = torch.empty((rows, inter // 32, Q8_1_BLOCK_BYTES), dtype=torch.uint8, device=gate.device)
+    if tuple(q8.shape) != (rows, inter // 32, Q8_1_BLOCK_BYTES) or q8.dtype != torch.uint8 or \
+            not q8.is_contiguous() or q8.device != gate.device:
+        raise ValueError(f"q8 must be a contiguous uint8 CUDA tensor [{rows}, {inter // 32}, 36]")
+    wp = None
+    if w is not None:
+        if tuple(w.shape) != (rows,) or w.dtype != torch.float32 or not w.is_contiguous() or \
+                w.device != gate.device:
+            raise ValueError(f"w must be a contiguous float32 CUDA tensor [{rows}]")
+        wp = w.data_ptr()
+    with torch.cuda.device(gate.device):
+        stream = torch.cuda.current_stream(gate.device).cuda_stream
+        sdq_swiglu_q8_1(gate.data_ptr(), ld_g, up.data_ptr(), ld_u, wp, h.data_ptr(), ld_h,
+                        q8.data_ptr(), rows, inter, limit, stream)
+    return h, q8
 
 
 def run(x: torch.Tensor, grad_y: torch.Tensor, group_size: int = GROUP_SIZE, codes: str = "int8",

@@ -37,6 +37,10 @@ _lib.sdq_fuse_strided.argtypes = _STRIDED + [_P]
 _lib.sdq_fuse_strided.restype = ctypes.c_int
 _lib.sdq_validate_strided.argtypes = _STRIDED
 _lib.sdq_validate_strided.restype = ctypes.c_int
+_lib.sdq_swiglu_q8_1.argtypes = [_P, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _I64, ctypes.c_float, _P]
+_lib.sdq_swiglu_q8_1.restype = ctypes.c_int
+_lib.sdq_validate_swiglu_q8_1.argtypes = [_P, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _I64]
+_lib.sdq_validate_swiglu_q8_1.restype = ctypes.c_int
 _lib.sdq_fuse_host.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P, ctypes.c_size_t, _I64, _P]
 _lib.sdq_fuse_host.restype = ctypes.c_int
 _lib.sdq_fuse_host_workspace_bytes.argtypes = [_I64, _I64, _I64]
@@ -138,6 +142,21 @@ def sdq_validate_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: i
     return int(_lib.sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
                                          ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t,
                                          ld_y_q_t, y_s_t, ld_y_s_t, M, K, group_size, format))
+
+
+def sdq_swiglu_q8_1(gate: int, ld_gate: int, up: int, ld_up: int, w: Optional[int], h: int, ld_h: int,
+                    q8: int, rows: int, inter: int, limit: float = 0.0,
+                    stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the forward SwiGLU + q8_1 entry point (w may be None)."""
+    _check(_lib.sdq_swiglu_q8_1(gate, ld_gate, up, ld_up, w or None, h, ld_h, q8, rows, inter,
+                                float(limit), stream or 0), "sdq_swiglu_q8_1")
+
+
+def sdq_validate_swiglu_q8_1(gate: int, ld_gate: int, up: int, ld_up: int, w: Optional[int], h: int,
+                             ld_h: int, q8: int, rows: int, inter: int) -> int:
+    """Argument checks of sdq_swiglu_q8_1 only (no CUDA call); returns the status code."""
+    return int(_lib.sdq_validate_swiglu_q8_1(gate, ld_gate, up, ld_up, w or None, h, ld_h, q8, rows,
+                                             inter))
 
 
 def sdq_validate_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y_q_t: int,

@@ -4,7 +4,8 @@
 
 (run it as a script: importing the package needs the library it builds)
 
-nvcc compiles ``csrc/sdq_api.cu`` (host API + the fused kernel) into a shared
+nvcc compiles ``csrc/sdq_api.cu`` (host API + the fused kernel) and
+``csrc/fwd_api.cu`` (the forward-side SwiGLU + q8_1 kernel) into a shared
 library with a C ABI (``include/sdq.h``); the CUDA runtime is linked
 statically and the driver's tensor-map encoder is looked up at run time, so
 the library needs only the NVIDIA driver at load time.
@@ -21,8 +22,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsdq.so")
-SOURCES = [os.path.join(CSRC, "sdq_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sdq_kernel.cuh", "sdq_ptx.cuh")] + [
+SOURCES = [os.path.join(CSRC, f) for f in ("sdq_api.cu", "fwd_api.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sdq_kernel.cuh", "sdq_ptx.cuh", "fwd_kernel.cuh")] + [
     os.path.join(INCLUDE, "sdq.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -63,6 +63,15 @@ int cuda_fail(cudaError_t e) {
   return SDQ_ERR_CUDA;
 }
 
+}  // namespace
+
+// Shared with the library's other translation units (fwd_api.cu).
+namespace sdq_internal {
+int cuda_fail(cudaError_t e) { return ::cuda_fail(e); }
+}  // namespace sdq_internal
+
+namespace {
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;

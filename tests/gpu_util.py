@@ -239,3 +239,83 @@ def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", gro
         assert not bad.any(), f"{where} {name}: {int(bad.sum())} values more than a step apart"
         assert nd <= 1e-3 * a.size, f"{where} {name}: {nd} of {a.size} codes differ"
     return stats
+
+
+# ---- the forward-side neighbour (SwiGLU forward + q8_1 rows) -----------------
+#
+# Tolerances, from the same arithmetic as the backward op: h = bf16 of an fp32
+# computation (hardware exp2/reciprocal approximations, two roundings before
+# bf16) against the oracle's fp64 value rounded once, so an h next to a bf16
+# rounding boundary can round the other way: h within one bf16 step, and equal
+# on all but 0.1 %; the codes within 1 (the kernel multiplies by 1/d32, the
+# oracle divides), equal on all but 0.1 %; d (fp16) within a relative 2^-7
+# (only a flipped amax moves it).  sum = fp16(d32 * sum(q)) is a function of
+# the block's d32 and codes, which the two checks above compare with the
+# oracle (a flipped amax moves d32 and, with it, up to every code of the
+# block by one), so the kernel's sum is checked against its own block:
+# |sum - d * sum(q)| within the fp16 rounding of d and of the product.
+
+def run_cuda_fwd(gate_u16, up_u16, w, limit=0.0, ld_pad=0):
+    """The forward entry on the device; gate/up may be views (row stride kept
+    if ld_pad is 0, else copied into rows padded by ld_pad elements); h and
+    q8 are guarded and prefilled.  Returns numpy (h uint16 [rows, inter],
+    q8 uint8 [rows, inter/32, 36])."""
+    import swiglu_backward_int8_b200 as sdq
+    rows, inter = gate_u16.shape
+
+    def dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        if ld_pad:
+            buf = torch.zeros((rows, inter + ld_pad), dtype=torch.bfloat16, device="cuda")
+            buf[:, :inter] = t
+            return buf[:, :inter]
+        return t
+
+    g, u = dev(gate_u16), dev(up_u16)
+    wd = torch.from_numpy(np.ascontiguousarray(w, np.float32)).cuda() if w is not None else None
+    hb = Guarded((rows, inter), torch.int16, -1)              # 0xFFFF: a NaN bf16, never written
+    qb = Guarded((rows, inter // 32, 36), torch.uint8, 0xA5)
+    sdq.swiglu_q8_1(g, u, wd, limit, hb.t.view(torch.bfloat16), qb.t)
+    torch.cuda.synchronize()
+    assert hb.guards_intact() and qb.guards_intact(), "guard bytes overwritten"
+    h = hb.t.cpu().numpy().view(np.uint16)
+    q8 = qb.t.cpu().numpy()
+    assert not (h == 0xFFFF).any(), "h left unwritten"
+    return h, q8
+
+
+def compare_fwd(got, ref, where=""):
+    h, q8 = got
+    rh, rq8 = ref
+    assert h.shape == rh.shape and q8.shape == rq8.shape
+    # h: bf16 bits as signed-magnitude ordinals
+    def ordv(b):
+        b = b.astype(np.int64)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+    dh = np.abs(ordv(h) - ordv(rh))
+    nh = int((h != rh).sum())
+    assert dh.max(initial=0) <= 1, f"{where} h: {dh.max()} bf16 steps apart"
+    assert nh <= 1e-3 * h.size, f"{where} h: {nh} of {h.size} differ"
+    q, rq = q8[..., 4:].view(np.int8).astype(np.int16), rq8[..., 4:].view(np.int8).astype(np.int16)
+    dq = np.abs(q - rq)
+    nq = int((dq != 0).sum())
+    assert dq.max(initial=0) <= 1, f"{where} codes: {dq.max()} apart"
+    assert nq <= 1e-3 * q.size, f"{where} codes: {nq} of {q.size} differ"
+    d = q8[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    rd = rq8[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    s = q8[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    rs = rq8[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    both_zero = (d == 0) & (rd == 0)
+    rel = np.where(both_zero, 0.0, np.abs(d - rd) / np.maximum(np.abs(rd), 1e-300))
+    assert rel.max(initial=0) <= 2.0 ** -7, f"{where} d: rel {rel.max()}"
+    ulp = lambda v: np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -14))).astype(int) - 10)
+    ds = np.abs(s - rs)
+    qsum = q.sum(axis=-1)
+    own = d * qsum                            # fp16 d is within half its spacing of d32
+    tol = np.abs(qsum) * ulp(d) / 2 + ulp(s) / 2 + np.abs(own) * 2.0 ** -40
+    bad = np.abs(s - own) > tol
+    assert not bad.any(), f"{where} sum: {int(bad.sum())} blocks off their own d * sum(q)"
+    same = (q == rq).all(axis=-1) & (d == rd)  # where the block agrees, the sum must too
+    assert np.array_equal(s[same], rs[same]), f"{where} sum differs on blocks that agree"
+    del ds
+    return {"h_n_diff": nh, "q_n_diff": nq, "d_n_diff": int((d != rd).sum()), "s_n_diff": int((s != rs).sum())}

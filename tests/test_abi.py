@@ -212,3 +212,13 @@ def test_wrapper_takes_row_strides_and_refuses_other_layouts():
               (torch.bfloat16,), True, torch.device("cpu"))
     with pytest.raises(ValueError):          # the host entry points need contiguous tensors
         _rows("x", wide[:, :512], (8, 512), (torch.bfloat16,), False, torch.device("cpu"))
+
+
+def test_fwd_rejects_bad_arguments_without_launching():
+    import swiglu_backward_int8_b200 as sdq
+    A = 1 << 20
+    assert sdq.sdq_validate_swiglu_q8_1(A, 64, A, 64, None, A, 64, A, 4, 48) == sdq.Status.ERR_SHAPE
+    assert sdq.sdq_validate_swiglu_q8_1(A, 60, A, 64, None, A, 64, A, 4, 64) == sdq.Status.ERR_STRIDE
+    assert sdq.sdq_validate_swiglu_q8_1(A + 2, 64, A, 64, None, A, 64, A, 4, 64) == sdq.Status.ERR_ALIGN
+    assert sdq.sdq_validate_swiglu_q8_1(A, 64, A, 64, None, A, 64, A + 2, 4, 64) == sdq.Status.ERR_ALIGN
+    assert sdq.sdq_validate_swiglu_q8_1(0, 64, 0, 64, None, 0, 64, 0, 0, 64) == sdq.Status.OK

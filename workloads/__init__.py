@@ -226,3 +226,23 @@ def small_workload(M: int, K: int, seed: int = 7, sigma_x: float = 1.0,
     """An ad-hoc shape with the same recipe (tests of odd and tiny shapes)."""
     return Workload(f"swiglu_bwd_int8_M{M}_K{K}_s{seed}", M, K, sigma_x,
                     sigma_grad_y, seed, **kw)
+
+
+# ---- the forward-side neighbour (SwiGLU forward + q8_1 rows) ------------------
+
+STREAM_ROW_WEIGHT = 7
+
+
+def row_weights(seed: int, rows: int) -> np.ndarray:
+    """Per-row weights (e.g. MoE router weights) uniform in (0, 1], float32,
+    from the seed's own stream."""
+    u = uniforms(stream_key(seed, STREAM_ROW_WEIGHT), 0, rows)
+    return (1.0 - u).astype(np.float32)
+
+
+def fwd_inputs(w: Workload):
+    """(gate, up, row weights) of a workload for the forward op: gate and up
+    are the two halves of the workload's x ([rows, K] bf16 bits each, as views
+    of x with row stride 2K), rows = M, inter = K."""
+    x, _ = make_inputs(w)
+    return x[:, :w.K], x[:, w.K:], row_weights(w.seed, w.M)
