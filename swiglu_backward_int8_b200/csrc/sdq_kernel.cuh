@@ -263,10 +263,19 @@ __device__ __forceinline__ void store_scale(void* base, int64_t idx, float scale
 // 1.5 * 2^23 inside the fused multiply-add rounds to an integer).  E4M3: the
 // two fp32 products.
 template <bool kE4M3, bool kTiny>
-__device__ __forceinline__ float2 quant2(uint32_t v, float2 inv, float2 pre) {
+__device__ __forceinline__ float2 quant2(uint32_t v, float2 inv, float2 pre, float2 scl) {
   float2 x = unpack2(v);
   if (kTiny) x = __fmul2_rn(x, pre);
-  if (kE4M3) return __fmul2_rn(x, inv);
+  if (kE4M3) {
+    // The quotient x / scale correctly rounded to fp32, from the reciprocal
+    // and one correction (Markstein): r = x * inv, then the exact remainder
+    // x - r * scale, then r + remainder * inv.  E4M3 keeps three mantissa
+    // bits, so x / scale often sits exactly on a rounding tie of the code,
+    // where the plain product could fall on either side.
+    const float2 r = __fmul2_rn(x, inv);
+    const float2 e = __ffma2_rn(make_float2(-r.x, -r.y), scl, x);
+    return __ffma2_rn(e, inv, r);
+  }
   return __ffma2_rn(x, inv, make_float2(12582912.0f, 12582912.0f));
 }
 
@@ -279,15 +288,18 @@ __device__ __forceinline__ uint32_t pack_codes(float2 a, float2 b) {
 }
 
 // Sixteen codes of one row piece (8 bf16 pairs) with one inverse scale.
+// `scale`: the group's scale (times kTinyPre for the tiny path), used by the
+// E4M3 quotient correction only.
 template <bool kE4M3, bool kTiny>
-__device__ __forceinline__ uint4 quant16(const uint32_t (&v)[8], float inv) {
+__device__ __forceinline__ uint4 quant16(const uint32_t (&v)[8], float inv, float scale) {
   const float2 iv = make_float2(inv, inv);
   const float2 pre = make_float2(kTinyPre, kTinyPre);
+  const float2 sc = make_float2(scale, scale);
   uint32_t w[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k)
-    w[k] = pack_codes<kE4M3>(quant2<kE4M3, kTiny>(v[2 * k], iv, pre),
-                             quant2<kE4M3, kTiny>(v[2 * k + 1], iv, pre));
+    w[k] = pack_codes<kE4M3>(quant2<kE4M3, kTiny>(v[2 * k], iv, pre, sc),
+                             quant2<kE4M3, kTiny>(v[2 * k + 1], iv, pre, sc));
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -295,10 +307,10 @@ __device__ __forceinline__ uint4 quant16(const uint32_t (&v)[8], float inv) {
 // 16-byte code rows (low channel, high channel).
 template <bool kE4M3, bool kTiny>
 __device__ __forceinline__ void quant_cols(const uint32_t (&v)[16], float2 inv, float2 pre,
-                                           uint4& lo, uint4& hi) {
+                                           float2 scl, uint4& lo, uint4& hi) {
   float2 q[16];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) q[t] = quant2<kE4M3, kTiny>(v[t], inv, pre);
+  for (int t = 0; t < 16; ++t) q[t] = quant2<kE4M3, kTiny>(v[t], inv, pre, scl);
   uint32_t wl[4], wh[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
@@ -387,10 +399,12 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   uint4 lo, hi;
   if (__any_sync(kFull, i_lo < 0.0f || i_hi < 0.0f)) {   // a tiny group in this warp (rare)
     // pre-multiply only the tiny channels; the others use factor 1
-    quant_cols<kE4M3, true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)),
-                            make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f), lo, hi);
+    const float2 pre = make_float2(i_lo < 0.0f ? kTinyPre : 1.0f, i_hi < 0.0f ? kTinyPre : 1.0f);
+    quant_cols<kE4M3, true>(v, make_float2(fabsf(i_lo), fabsf(i_hi)), pre,
+                            make_float2(s_lo * pre.x, s_hi * pre.y), lo, hi);
   } else {
-    quant_cols<kE4M3, false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), lo, hi);
+    quant_cols<kE4M3, false>(v, make_float2(i_lo, i_hi), make_float2(1.0f, 1.0f), make_float2(s_lo, s_hi),
+                             lo, hi);
   }
   const int tok = 16 * kc;
   if (tok < valid) {
@@ -573,11 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (r < valid) {
         uint4 og, ou;
         if (__any_sync(__activemask(), ig < 0.0f || iu < 0.0f)) {   // a tiny group in this warp (rare)
-          og = (ig < 0.0f) ? quant16<kE4M3, true>(dgp, -ig) : quant16<kE4M3, false>(dgp, ig);
-          ou = (iu < 0.0f) ? quant16<kE4M3, true>(dup, -iu) : quant16<kE4M3, false>(dup, iu);
+          og = (ig < 0.0f) ? quant16<kE4M3, true>(dgp, -ig, sg * kTinyPre) : quant16<kE4M3, false>(dgp, ig, sg);
+          ou = (iu < 0.0f) ? quant16<kE4M3, true>(dup, -iu, su * kTinyPre) : quant16<kE4M3, false>(dup, iu, su);
         } else {
-          og = quant16<kE4M3, false>(dgp, ig);
-          ou = quant16<kE4M3, false>(dup, iu);
+          og = quant16<kE4M3, false>(dgp, ig, sg);
+          ou = quant16<kE4M3, false>(dup, iu, su);
         }
         int8_t* dst = giq_t + r * p.ld_giq;
         st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));

@@ -199,7 +199,8 @@ def _scale_values(s, scales):
     return np.ldexp(1.0, s.astype(np.int64) - 127) if scales else s.astype(np.float64)
 
 
-def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", group_size: int = 128):
+def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", group_size: int = 128,
+                max_frac: float = 1e-3):
     """Assert the format tolerances; returns mismatch statistics."""
     giq, gis, yqt, yst = got
     rq, rs, ryq, rys = ref
@@ -237,7 +238,7 @@ def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", gro
         stats[name] = {"n_diff": nd, "frac_diff": nd / max(1, a.size), "n_out_of_step": int(bad.sum()),
                        "n_signed_zero": int(signed_zero.sum())}
         assert not bad.any(), f"{where} {name}: {int(bad.sum())} values more than a step apart"
-        assert nd <= 1e-3 * a.size, f"{where} {name}: {nd} of {a.size} codes differ"
+        assert nd <= max_frac * a.size, f"{where} {name}: {nd} of {a.size} codes differ"
     return stats
 
 

@@ -94,3 +94,48 @@ def test_formats_over_the_whole_exponent_range(fmt):
     gy = np.full((M, K), 0x3F80, np.uint16)             # 1.0
     w = W.small_workload(M, K, seed=0)
     _check(w, fmt, x, gy)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("fmt,G", [((1, 1, 1), 128), ((0, 0, 0), 64), ((1, 0, 0), 32)])
+def test_formats_full_size_sampled_tiles(fmt, G):
+    """M=16384, K=7168 in one launch (the bench's largest workload) in another
+    format or group size: 24 sampled 128x128 tiles against the format oracle
+    on each tile (every group lies inside one tile)."""
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    codes, scales, layout = fmt
+    w = W.WORKLOADS[4]
+    x, gy = W.make_inputs(w)
+    M, K = w.M, w.K
+    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
+    names = ("e4m3" if codes else "int8", "e8m0" if scales else "fp32", "mg_k" if layout else "k_mg")
+    outs = sdq.allocate_outputs(M, K, "cuda", G, *names)
+    sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *outs, group_size=G, codes=names[0], scales=names[1],
+                                    y_scale_layout=names[2])
+    torch.cuda.synchronize()
+    assert sdq.sdq_device_status() == 0
+    giq, gis, yqt, yst = (t.view(torch.uint8).cpu().numpy() if t.dtype != torch.float32 else t.cpu().numpy()
+                          for t in outs)
+    if layout:
+        yst = yst.T
+    rng = np.random.default_rng(7)
+    tiles = {(0, 0), (M // 128 - 1, K // 128 - 1)}
+    while len(tiles) < 24:
+        tiles.add((int(rng.integers(M // 128)), int(rng.integers(K // 128))))
+    per = 128 // G
+    n_diff = 0
+    for i, j in sorted(tiles):
+        r0, c0 = 128 * i, 128 * j
+        xt = np.concatenate([x[r0:r0 + 128, c0:c0 + 128], x[r0:r0 + 128, K + c0:K + c0 + 128]], axis=1)
+        ref = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(xt, gy[r0:r0 + 128, c0:c0 + 128], G, codes, scales, 0)
+        got = (np.concatenate([giq[r0:r0 + 128, c0:c0 + 128], giq[r0:r0 + 128, K + c0:K + c0 + 128]], axis=1),
+               np.concatenate([gis[r0:r0 + 128, j * per:(j + 1) * per],
+                               gis[r0:r0 + 128, K // G + j * per:K // G + (j + 1) * per]], axis=1),
+               yqt[c0:c0 + 128, r0:r0 + 128], yst[c0:c0 + 128, i * per:(i + 1) * per])
+        st = U.compare_fmt(got, ref, codes, scales, 0, f"M16384 tile ({i},{j}) {fmt} G={G}", G,
+                           max_frac=1.0)                 # the 0.1 % bound applies to the whole sample
+        for name in ("grad_input_q", "y_q_t"):
+            n_diff += st[name]["n_diff"]
+    total = 24 * 128 * 128 * 3
+    assert n_diff <= 1e-3 * total, f"{n_diff} of {total} sampled codes differ"
