@@ -15,7 +15,8 @@
 // of one row (8 blocks); a lane holds 8 of them (one 16-byte load of gate and
 // of up, one 16-byte store of h), so a block is 4 neighbouring lanes and its
 // amax and code sum take two shuffles.  A persistent grid walks the
-// (row, 256-element chunk) units.
+// (row, 256-element chunk) units, two per warp iteration (both units' loads
+// in flight before either is computed).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -88,84 +89,124 @@ __device__ __forceinline__ void swiglu8(const uint4& g, const uint4& u, float w,
   }
 }
 
+// One warp unit after its loads: h, its store, and the unit's 8 q8_1 blocks.
+// tab: per bf16 mantissa m, (fl((1 + m/128)/127), its reciprocal); for a
+// block amax (1 + m/128) * 2^e with a bf16 exponent field >= 10 the scale
+// fl(amax/127) and 1/scale are those entries with 2^e moved into the
+// exponent fields, exactly (both stay normal floats).
+__device__ __forceinline__ void finish_unit(const Params& p, const float2* tab, const uint4& g,
+                                            const uint4& u, float w, int64_t m, int k0, bool active,
+                                            int lane) {
+  constexpr unsigned kFull = 0xffffffffu;
+  uint32_t h[4] = {0u, 0u, 0u, 0u};
+  if (active) {
+    swiglu8(g, u, w, p, h);
+    st_cs_v4(reinterpret_cast<int8_t*>(p.h + 2 * (m * p.ld_h + k0)), make_uint4(h[0], h[1], h[2], h[3]));
+  }
+  // block amax over the 4 lanes of the block (bf16, exact)
+  uint32_t a = absmax_bf16x2(absmax_bf16x2(h[0], h[1]), absmax_bf16x2(h[2], h[3]));
+  a = absmax_bf16x2(a, __shfl_xor_sync(kFull, a, 1));
+  a = absmax_bf16x2(a, __shfl_xor_sync(kFull, a, 2));
+  const uint32_t ab = (a & 0x7FFFu) > ((a >> 16) & 0x7FFFu) ? (a & 0x7FFFu) : ((a >> 16) & 0x7FFFu);
+  float d = 0.0f;
+  uint32_t qw[2] = {0u, 0u};
+  int qs = 0;
+  if (ab >= 0x0500u) {   // amax >= 2^-117: the table path, then multiply by 1/d32
+    const float2 t = tab[ab & 127u];
+    const int sh = (static_cast<int>(ab >> 7) - 127) << 23;
+    d = __int_as_float(__float_as_int(t.x) + sh);
+    const float inv = __int_as_float(__float_as_int(t.y) - sh);
+    const float2 iv = make_float2(inv, inv);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float2 q0 = __ffma2_rn(bf2(h[2 * c]), iv, magic);
+      const float2 q1 = __ffma2_rn(bf2(h[2 * c + 1]), iv, magic);
+      qw[c] = pack_low_bytes(__float_as_uint(q0.x), __float_as_uint(q0.y), __float_as_uint(q1.x),
+                             __float_as_uint(q1.y));
+      qs += (static_cast<int>(__float_as_uint(q0.x)) - 0x4B400000) +
+            (static_cast<int>(__float_as_uint(q0.y)) - 0x4B400000) +
+            (static_cast<int>(__float_as_uint(q1.x)) - 0x4B400000) +
+            (static_cast<int>(__float_as_uint(q1.y)) - 0x4B400000);
+    }
+  } else if (ab != 0u) {  // tiny block (1/d32 may overflow): divide, as the definition reads
+    d = __fdiv_rn(__uint_as_float(ab << 16), 127.0f);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      int qb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t pr = h[2 * c + (e >> 1)];
+        const float v = (e & 1) ? bf16_hi(pr) : bf16_lo(pr);
+        qb[e] = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v, d)), -127.0f), 127.0f));
+        qs += qb[e];
+      }
+      qw[c] = (qb[0] & 0xFF) | ((qb[1] & 0xFF) << 8) | ((qb[2] & 0xFF) << 16) |
+              (static_cast<uint32_t>(qb[3] & 0xFF) << 24);
+    }
+  }
+  qs += __shfl_xor_sync(kFull, qs, 1);
+  qs += __shfl_xor_sync(kFull, qs, 2);
+  if (active) {
+    uint8_t* b = p.q8 + (m * (p.inter / kBlock) + k0 / kBlock) * kBlockBytes;
+    const int part = lane & 3;                          // 8 codes at bytes 4 + 8 * part
+    *reinterpret_cast<uint32_t*>(b + 4 + 8 * part) = qw[0];
+    *reinterpret_cast<uint32_t*>(b + 8 + 8 * part) = qw[1];
+    if (part == 0) {   // an all-zero block has d = 0 and qs = 0: both halves 0
+      const __half dh = __float2half_rn(d);
+      const __half sh = __double2half(static_cast<double>(d) * static_cast<double>(qs));
+      *reinterpret_cast<uint32_t*>(b) = static_cast<uint32_t>(__half_as_ushort(dh)) |
+                                        (static_cast<uint32_t>(__half_as_ushort(sh)) << 16);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
     swiglu_q8_1_kernel(const Params p) {
-  constexpr unsigned kFull = 0xffffffffu;
+  __shared__ float2 tab[128];
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 128) {
+    const float t = __fdiv_rn(1.0f + static_cast<float>(threadIdx.x) * (1.0f / 128.0f), 127.0f);
+    tab[threadIdx.x] = make_float2(t, __frcp_rn(t));
+  }
+  __syncthreads();
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
   const int64_t units = p.rows * p.units_per_row;
-  const int nblk_row = p.inter / kBlock;
+  // The warp's units are warp0, warp0 + nwarps, ...; (row, chunk) of the next
+  // one is (row, chunk) + (dm, dc) with a carry, so no division per unit.
+  const int upr = p.units_per_row;
+  int64_t m = warp0 / upr;
+  int c = static_cast<int>(warp0 - m * upr);
+  const int64_t dm = nwarps / upr;
+  const int dc = static_cast<int>(nwarps - dm * upr);
   grid_dependency_wait();   // inputs may come from the previous kernel in the stream
   grid_launch_dependents();
-  for (int64_t unit = warp0; unit < units; unit += nwarps) {
-    const int64_t m = unit / p.units_per_row;
-    const int chunk = static_cast<int>(unit - m * p.units_per_row);
-    const int k0 = chunk * kUnit + lane * 8;           // this lane's first element
-    const bool active = k0 < p.inter;                  // whole blocks: inter % 32 == 0
-    uint32_t h[4] = {0u, 0u, 0u, 0u};
-    if (active) {
-      const uint4 g = *reinterpret_cast<const uint4*>(p.gate + 2 * (m * p.ld_gate + k0));
-      const uint4 u = *reinterpret_cast<const uint4*>(p.up + 2 * (m * p.ld_up + k0));
-      const float w = p.w ? p.w[m] : 1.0f;
-      swiglu8(g, u, w, p, h);
-      st_cs_v4(reinterpret_cast<int8_t*>(p.h + 2 * (m * p.ld_h + k0)), make_uint4(h[0], h[1], h[2], h[3]));
+  // two units per iteration: both units' loads are in flight before either is computed
+  for (int64_t unit = warp0; unit < units; unit += 2 * nwarps) {
+    int64_t m1 = m + dm;
+    int c1 = c + dc;
+    if (c1 >= upr) { c1 -= upr; ++m1; }
+    const bool has1 = unit + nwarps < units;            // warp-uniform
+    const int k0 = c * kUnit + lane * 8, k1 = c1 * kUnit + lane * 8;
+    const bool act0 = k0 < p.inter, act1 = has1 && k1 < p.inter;   // whole blocks: inter % 32 == 0
+    uint4 g0 = make_uint4(0, 0, 0, 0), u0 = g0, g1 = g0, u1 = g0;
+    float w0 = 1.0f, w1 = 1.0f;
+    if (act0) {
+      g0 = *reinterpret_cast<const uint4*>(p.gate + 2 * (m * p.ld_gate + k0));
+      u0 = *reinterpret_cast<const uint4*>(p.up + 2 * (m * p.ld_up + k0));
+      if (p.w) w0 = p.w[m];
     }
-    // block amax over the 4 lanes of the block (bf16, exact)
-    uint32_t a = absmax_bf16x2(absmax_bf16x2(h[0], h[1]), absmax_bf16x2(h[2], h[3]));
-    a = absmax_bf16x2(a, __shfl_xor_sync(kFull, a, 1));
-    a = absmax_bf16x2(a, __shfl_xor_sync(kFull, a, 2));
-    const uint32_t ab = (a & 0x7FFFu) > ((a >> 16) & 0x7FFFu) ? (a & 0x7FFFu) : ((a >> 16) & 0x7FFFu);
-    const float amax = __uint_as_float(ab << 16);
-    const float d = __fdiv_rn(amax, 127.0f);
-    uint32_t qw[2] = {0u, 0u};
-    int qs = 0;
-    if (ab >= 0x0500u) {   // amax >= 2^-117: d32 and 1/d32 are normal floats, multiply by 1/d32
-      const float inv = __frcp_rn(d);
-      const float2 iv = make_float2(inv, inv);
-      const float2 magic = make_float2(12582912.0f, 12582912.0f);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const float2 q0 = __ffma2_rn(bf2(h[2 * c]), iv, magic);
-        const float2 q1 = __ffma2_rn(bf2(h[2 * c + 1]), iv, magic);
-        qw[c] = pack_low_bytes(__float_as_uint(q0.x), __float_as_uint(q0.y), __float_as_uint(q1.x),
-                               __float_as_uint(q1.y));
-        qs += (static_cast<int>(__float_as_uint(q0.x)) - 0x4B400000) +
-              (static_cast<int>(__float_as_uint(q0.y)) - 0x4B400000) +
-              (static_cast<int>(__float_as_uint(q1.x)) - 0x4B400000) +
-              (static_cast<int>(__float_as_uint(q1.y)) - 0x4B400000);
-      }
-    } else if (ab != 0u) {  // tiny block (1/d32 may overflow): divide, as the definition reads
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        int qb[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t pr = h[2 * c + (e >> 1)];
-          const float v = (e & 1) ? bf16_hi(pr) : bf16_lo(pr);
-          qb[e] = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v, d)), -127.0f), 127.0f));
-          qs += qb[e];
-        }
-        qw[c] = (qb[0] & 0xFF) | ((qb[1] & 0xFF) << 8) | ((qb[2] & 0xFF) << 16) |
-                (static_cast<uint32_t>(qb[3] & 0xFF) << 24);
-      }
+    if (act1) {
+      g1 = *reinterpret_cast<const uint4*>(p.gate + 2 * (m1 * p.ld_gate + k1));
+      u1 = *reinterpret_cast<const uint4*>(p.up + 2 * (m1 * p.ld_up + k1));
+      if (p.w) w1 = p.w[m1];
     }
-    qs += __shfl_xor_sync(kFull, qs, 1);
-    qs += __shfl_xor_sync(kFull, qs, 2);
-    if (active) {
-      const int blk = k0 / kBlock;
-      uint8_t* b = p.q8 + (m * nblk_row + blk) * kBlockBytes;
-      const int part = lane & 3;                          // 8 codes at bytes 4 + 8 * part
-      *reinterpret_cast<uint32_t*>(b + 4 + 8 * part) = qw[0];
-      *reinterpret_cast<uint32_t*>(b + 8 + 8 * part) = qw[1];
-      if (part == 0) {
-        const __half dh = __float2half_rn(ab ? d : 0.0f);
-        const __half sh = __double2half(static_cast<double>(d) * static_cast<double>(qs));
-        const uint32_t ds = static_cast<uint32_t>(__half_as_ushort(dh)) |
-                            (static_cast<uint32_t>(__half_as_ushort(ab ? sh : __float2half_rn(0.0f))) << 16);
-        *reinterpret_cast<uint32_t*>(b) = ds;
-      }
-    }
+    finish_unit(p, tab, g0, u0, w0, m, k0, act0, lane);
+    if (has1) finish_unit(p, tab, g1, u1, w1, m1, k1, act1, lane);
+    m = m1 + dm;
+    c = c1 + dc;
+    if (c >= upr) { c -= upr; ++m; }
   }
 }
 
