@@ -76,8 +76,10 @@ def run_cuda(x_u16: np.ndarray, gy_u16: np.ndarray, stream=None):
     return giq, gis, yqt, yst
 
 
-def compare(got, ref, where=""):
-    """Assert the tolerances; returns mismatch statistics."""
+def compare(got, ref, where="", max_frac=INT8_MAX_FRAC):
+    """Assert the tolerances; returns mismatch statistics.  max_frac: the
+    bound on the fraction of differing codes (a sampled test applies it to
+    the whole sample instead)."""
     giq, gis, yqt, yst = got
     rq, rs, ryq, rys = ref
     stats = {}
@@ -88,7 +90,7 @@ def compare(got, ref, where=""):
         stats[name] = {"max_abs_diff": int(d.max()) if d.size else 0, "n_diff": nd,
                        "frac_diff": nd / max(1, d.size)}
         assert d.max(initial=0) <= INT8_MAX_DIFF, f"{where} {name}: max |dq| = {d.max()}"
-        assert nd <= INT8_MAX_FRAC * d.size, f"{where} {name}: {nd} of {d.size} differ"
+        assert nd <= max_frac * d.size, f"{where} {name}: {nd} of {d.size} differ"
     for name, a, b in (("grad_input_s", gis, rs), ("y_s_t", yst, rys)):
         assert a.shape == b.shape, (name, a.shape, b.shape)
         rel = np.abs(a.astype(np.float64) - b.astype(np.float64)) / np.abs(b.astype(np.float64))

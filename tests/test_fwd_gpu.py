@@ -78,3 +78,12 @@ def test_fwd_gates_below_the_fp32_sigmoid_range():
     h, _ = U.run_cuda_fwd(g, u, wt)
     assert (h & 0x7FFF).astype(bool).sum() > inter      # many nonzero h where fp32 sigma underflows
     del st
+
+
+@pytest.mark.slow
+def test_fwd_maximum_inter_sampled_rows():
+    """inter = 2^20 (the largest accepted) on a few rows; rows are independent,
+    so the oracle runs on every row here."""
+    w = W.small_workload(3, 1 << 20, seed=98)
+    g, u, wt = W.fwd_inputs(w)
+    _check(g, u, wt, 0.0, "inter 2^20")
