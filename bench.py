@@ -110,13 +110,13 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, sources=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = kernel_sha()
+    sha = kernel_sha(sources)
     for line in open(path):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload and parts[1] == sha:
@@ -574,7 +574,8 @@ def run_fwd(args):
                        "l2": f"inputs+outputs rotate over {nsets} buffer sets (>= 3x L2)",
                        "timing": "K calls replayed from CUDA graphs, CUDA events"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": recorded_traffic(w.name + "_swiglu_q8_1", FWD_SOURCES),
                          "algorithmic_bytes_per_launch": nbytes, "kernel": "sdq::fwd::swiglu_q8_1_kernel"},
             "cpu_baseline": cpu,
             "e2e": {"unavailable": "the forward op has a device entry point only"},
