@@ -77,6 +77,8 @@ def parse_args():
                     help="fuse: the backward op (the headline); swiglu_q8_1: the forward-side "
                          "SwiGLU + q8_1 rows on the workload's gate and up (rows = M, inter = K)")
     ap.add_argument("--limit", type=float, default=0.0, help="swiglu_q8_1: the clamp (0: none)")
+    ap.add_argument("--with-y", action="store_true",
+                    help="also time the call with the optional bf16 y output")
     ap.add_argument("--all-formats", action="store_true",
                     help="also time every output format on the workload and add a per_format list")
     a = ap.parse_args()
@@ -283,12 +285,13 @@ def scale_bytes(fmt) -> int:
     return 1 if fmt[1] == "e8m0" else 4
 
 
-def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, fmt=PAGE_FORMAT):
+def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, fmt=PAGE_FORMAT,
+                   with_y: bool = False):
     import torch
     import swiglu_backward_int8_b200 as sdq
     M, K = w.M, w.K
     codes, scales, layout = fmt
-    footprint = w.algorithmic_bytes(scale_bytes(fmt))
+    footprint = w.algorithmic_bytes(scale_bytes(fmt)) + (2 * M * K if with_y else 0)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nsets = max(1, -(-3 * l2 // footprint))
     x0, g0 = _to_device_bf16(x_np, device), _to_device_bf16(gy_np, device)
@@ -297,13 +300,14 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
         xs = x0 if s == 0 else x0.clone()
         gs = g0 if s == 0 else g0.clone()
         sets.append((xs, gs, sdq.allocate_outputs(M, K, device, codes=codes, scales=scales,
-                                                  y_scale_layout=layout)))
+                                                  y_scale_layout=layout),
+                     torch.empty(M, K, dtype=torch.bfloat16, device=device) if with_y else None))
     stream = torch.cuda.current_stream(device)
 
     def call(k):
-        xs, gs, outs = sets[k % nsets]
+        xs, gs, outs, ys = sets[k % nsets]
         sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, codes=codes, scales=scales,
-                                        y_scale_layout=layout)
+                                        y_scale_layout=layout, y=ys)
 
     for k in range(warmup):
         call(k)
@@ -438,6 +442,16 @@ def run_sdq(args):
                                     "frac_of_measured_hbm": gbs / peak,
                                     "algorithmic_bytes_per_launch": fb})
 
+    with_y = None
+    if args.with_y:   # the same call also writing the optional bf16 y
+        yms, _, _ = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, with_y=True)
+        yms = parallel.max_over_ranks(yms, device)
+        us = yms / args.steps * 1e3
+        yb = w.algorithmic_bytes() + 2 * w.M * w.K
+        gbs = yb / (us * 1e-6) / 1e9
+        with_y = {"us_per_call": us, "GB_s": gbs, "frac_of_measured_hbm": gbs / peak,
+                  "algorithmic_bytes_per_launch": yb, "format": format_name(PAGE_FORMAT)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0)
@@ -466,6 +480,8 @@ def run_sdq(args):
             line["per_workload"] = per
         if per_fmt is not None:
             line["per_format"] = per_fmt
+        if with_y is not None:
+            line["with_y"] = with_y
         print(json.dumps(line), flush=True)
     import torch.distributed as tdist
     if tdist.is_initialized():

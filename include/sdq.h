@@ -170,6 +170,13 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
  *                      of 16 takes 16-byte stores, others byte stores)
  *   y_s_t              [K, ceil(M/group_size)] (or [ceil(M/group_size), K]
  *                      with SDQ_FMT_YS_MG_K) scales
+ *   y                  optional (NULL: not written, ld_y ignored): the
+ *                      recomputed y itself, bf16 [M, K], the very values
+ *                      y_q_t quantizes (e.g. for an fp32-accumulated check of
+ *                      the GEMM that consumes y_q_t); 16-byte aligned, ld a
+ *                      multiple of 8, K <= ld <= SDQ_MAX_LD.  The page
+ *                      ("outputs" section) lists no such output; it serves
+ *                      the step after the op.
  *   M, K, group_size, format, stream: as sdq_fuse_format.
  * Inputs may overlap each other (gate and up often do: two halves of one
  * buffer); outputs must not overlap inputs or each other.  SDQ_ERR_STRIDE
@@ -179,16 +186,16 @@ int sdq_fuse_strided(const void* gate, int64_t ld_gate, const void* up, int64_t 
                      const void* grad_y, int64_t ld_grad_y, void* grad_input_q,
                      int64_t ld_grad_input_q, void* grad_input_s, int64_t ld_grad_input_s,
                      void* y_q_t, int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t,
-                     int64_t M, int64_t K, int32_t group_size, uint32_t format,
-                     void* stream);
+                     void* y, int64_t ld_y, int64_t M, int64_t K, int32_t group_size,
+                     uint32_t format, void* stream);
 
 /* The argument checks of sdq_fuse_strided alone: no CUDA call, no launch. */
 int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
                          const void* grad_y, int64_t ld_grad_y, const void* grad_input_q,
                          int64_t ld_grad_input_q, const void* grad_input_s,
                          int64_t ld_grad_input_s, const void* y_q_t, int64_t ld_y_q_t,
-                         const void* y_s_t, int64_t ld_y_s_t, int64_t M, int64_t K,
-                         int32_t group_size, uint32_t format);
+                         const void* y_s_t, int64_t ld_y_s_t, const void* y, int64_t ld_y,
+                         int64_t M, int64_t K, int32_t group_size, uint32_t format);
 
 /*
  * sdq_swiglu_q8_1 -- the forward-side neighbour of the backward op: the

@@ -136,28 +136,38 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", s
     return M, K, ld_x, ld_gy, lds
 
 
-def _call_strided(gate, ld_gate, up, ld_up, grad_y, ld_gy, outs, lds, M, K, group_size, fmt, device):
+def _check_y(y, M, K, device):
+    """The optional bf16 y output: (pointer or None, leading dimension)."""
+    if y is None:
+        return None, 0
+    return y.data_ptr(), _rows("y", y, (M, K), (torch.bfloat16,), True, device)
+
+
+def _call_strided(gate, ld_gate, up, ld_up, grad_y, ld_gy, outs, lds, M, K, group_size, fmt, device,
+                  y=None):
+    yp, ld_y = _check_y(y, M, K, device)
     with torch.cuda.device(device):
         stream = torch.cuda.current_stream(device).cuda_stream
         q, s, yq, ys = outs
         sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y.data_ptr(), ld_gy, q.data_ptr(), lds[0],
-                         s.data_ptr(), lds[1], yq.data_ptr(), lds[2], ys.data_ptr(), lds[3], M, K,
-                         group_size, fmt, stream)
+                         s.data_ptr(), lds[1], yq.data_ptr(), lds[2], ys.data_ptr(), lds[3], yp,
+                         ld_y, M, K, group_size, fmt, stream)
 
 
 def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_input_q: torch.Tensor,
                                 grad_input_s: torch.Tensor, y_q_t: torch.Tensor,
                                 y_s_t: torch.Tensor, group_size: int = GROUP_SIZE, *,
                                 codes: Optional[str] = None, scales: Optional[str] = None,
-                                y_scale_layout: str = "k_mg") -> None:
+                                y_scale_layout: str = "k_mg", y: Optional[torch.Tensor] = None) -> None:
     """Fused SwiGLU backward + dual-axis quantization, in place, on the
     current CUDA stream of x's device.  The code format ("int8" or "e4m3")
     and the scale format ("fp32" or "e8m0") follow the dtypes of
     grad_input_q and grad_input_s unless given; ``y_scale_layout`` is "k_mg"
     (y_s_t [K, ceil(M/G)]) or "mg_k"; ``group_size`` is 128, 64 or 32.  Every
     tensor is 2-D row-major; rows may be padded (a slice of a wider buffer):
-    the library takes each tensor's row stride.  Raises ValueError on bad
-    arguments and SdqError on a library status."""
+    the library takes each tensor's row stride.  ``y`` (bf16 [M, K], optional)
+    also receives the recomputed y itself, the values y_q_t quantizes.
+    Raises ValueError on bad arguments and SdqError on a library status."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
     codes = _infer("codes", codes, grad_input_q, _CODE_DTYPES)
     scales = _infer("scales", scales, grad_input_s, _SCALE_DTYPES)
@@ -165,7 +175,7 @@ def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_inpu
     M, K, ld_x, ld_gy, lds = _check_tensors(x, grad_y, outs, group_size, True, codes, scales,
                                             y_scale_layout)
     _call_strided(x.data_ptr(), ld_x, x.data_ptr() + 2 * K, ld_x, grad_y, ld_gy, outs, lds, M, K,
-                  group_size, fmt, x.device)
+                  group_size, fmt, x.device, y)
 
 
 def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad_y: torch.Tensor,
@@ -173,7 +183,8 @@ def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad
                                       y_q_t: torch.Tensor, y_s_t: torch.Tensor,
                                       group_size: int = GROUP_SIZE, *, codes: Optional[str] = None,
                                       scales: Optional[str] = None,
-                                      y_scale_layout: str = "k_mg") -> None:
+                                      y_scale_layout: str = "k_mg",
+                                      y: Optional[torch.Tensor] = None) -> None:
     """The op with gate and up as two [M, K] bf16 tensors instead of one
     x = [gate | up] (e.g. the two halves of a fused projection kept apart);
     otherwise as silu_dot_fwd_bwd_quant_fuse."""
@@ -191,7 +202,7 @@ def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad
     ld_gy = _rows("grad_y", grad_y, (M, K), bf16, True, gate.device)
     lds = _check_outputs(M, K, outs, group_size, True, codes, scales, y_scale_layout, gate.device)
     _call_strided(gate.data_ptr(), ld_g, up.data_ptr(), ld_u, grad_y, ld_gy, outs, lds, M, K,
-                  group_size, fmt, gate.device)
+                  group_size, fmt, gate.device, y)
 
 
 def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,

@@ -32,7 +32,7 @@ _lib.sdq_fuse_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctype
 _lib.sdq_fuse_format.restype = ctypes.c_int
 _lib.sdq_validate_format.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, ctypes.c_uint32]
 _lib.sdq_validate_format.restype = ctypes.c_int
-_STRIDED = [_P, _I64] * 7 + [_I64, _I64, _I32, ctypes.c_uint32]
+_STRIDED = [_P, _I64] * 8 + [_I64, _I64, _I32, ctypes.c_uint32]
 _lib.sdq_fuse_strided.argtypes = _STRIDED + [_P]
 _lib.sdq_fuse_strided.restype = ctypes.c_int
 _lib.sdq_validate_strided.argtypes = _STRIDED
@@ -125,23 +125,27 @@ def sdq_fuse_format(x: int, grad_y: int, grad_input_q: int, grad_input_s: int, y
 
 def sdq_fuse_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: int, ld_grad_y: int,
                      grad_input_q: int, ld_grad_input_q: int, grad_input_s: int, ld_grad_input_s: int,
-                     y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int, M: int, K: int,
-                     group_size: int = 128, format: int = 0, stream: Optional[int] = None) -> None:
-    """Raw-pointer form of the strided entry point (leading dimensions in elements)."""
+                     y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int, y: Optional[int],
+                     ld_y: int, M: int, K: int, group_size: int = 128, format: int = 0,
+                     stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the strided entry point (leading dimensions in
+    elements; y, the optional bf16 y output, may be None)."""
     _check(_lib.sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
                                  ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t,
-                                 y_s_t, ld_y_s_t, M, K, group_size, format, stream or 0),
+                                 y_s_t, ld_y_s_t, y, ld_y, M, K, group_size, format, stream or 0),
            "sdq_fuse_strided")
 
 
 def sdq_validate_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: int, ld_grad_y: int,
                          grad_input_q: int, ld_grad_input_q: int, grad_input_s: int,
                          ld_grad_input_s: int, y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int,
-                         M: int, K: int, group_size: int = 128, format: int = 0) -> int:
+                         y: Optional[int], ld_y: int, M: int, K: int, group_size: int = 128,
+                         format: int = 0) -> int:
     """Argument checks of sdq_fuse_strided only (no CUDA call); returns the status code."""
     return int(_lib.sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
                                          ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t,
-                                         ld_y_q_t, y_s_t, ld_y_s_t, M, K, group_size, format))
+                                         ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y, M, K, group_size,
+                                         format))
 
 
 def sdq_swiglu_q8_1(gate: int, ld_gate: int, up: int, ld_up: int, w: Optional[int], h: int, ld_h: int,

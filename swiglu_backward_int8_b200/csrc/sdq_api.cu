@@ -24,34 +24,37 @@ constexpr int kStages = SDQ_STAGES;
 
 constexpr int kMaxDevices = 64;
 
-// One kernel per group size (32, 64, 128) and output format (SDQ_FMT_* bits 0..2).
+// One kernel per group size (32, 64, 128), output format (SDQ_FMT_* bits
+// 0..2) and whether bf16 y is written too.
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const sdq::Params);
 constexpr int kFormats = 8;
-constexpr int kKernels = 3 * kFormats;
+constexpr int kKernels = 2 * 3 * kFormats;
 
-template <int G>
+template <int G, bool kY>
 constexpr KernelFn kernel_of(int f) {
   switch (f) {
-    case 0: return sdq::fuse_kernel<kStages, G, false, false, false>;
-    case 1: return sdq::fuse_kernel<kStages, G, true, false, false>;
-    case 2: return sdq::fuse_kernel<kStages, G, false, true, false>;
-    case 3: return sdq::fuse_kernel<kStages, G, true, true, false>;
-    case 4: return sdq::fuse_kernel<kStages, G, false, false, true>;
-    case 5: return sdq::fuse_kernel<kStages, G, true, false, true>;
-    case 6: return sdq::fuse_kernel<kStages, G, false, true, true>;
-    default: return sdq::fuse_kernel<kStages, G, true, true, true>;
+    case 0: return sdq::fuse_kernel<kStages, G, false, false, false, kY>;
+    case 1: return sdq::fuse_kernel<kStages, G, true, false, false, kY>;
+    case 2: return sdq::fuse_kernel<kStages, G, false, true, false, kY>;
+    case 3: return sdq::fuse_kernel<kStages, G, true, true, false, kY>;
+    case 4: return sdq::fuse_kernel<kStages, G, false, false, true, kY>;
+    case 5: return sdq::fuse_kernel<kStages, G, true, false, true, kY>;
+    case 6: return sdq::fuse_kernel<kStages, G, false, true, true, kY>;
+    default: return sdq::fuse_kernel<kStages, G, true, true, true, kY>;
   }
 }
 
-// Kernel number n = 8 * (0, 1, 2 for group size 32, 64, 128) + format bits.
+// Kernel number n = 24 * (y written) + 8 * (0, 1, 2 for group size 32, 64, 128) + format bits.
 KernelFn kernel_at(int n) {
-  const int f = n % kFormats;
-  return n < kFormats ? kernel_of<32>(f) : n < 2 * kFormats ? kernel_of<64>(f) : kernel_of<128>(f);
+  const bool y = n >= 3 * kFormats;
+  const int g = (n % (3 * kFormats)) / kFormats, f = n % kFormats;
+  if (y) return g == 0 ? kernel_of<32, true>(f) : g == 1 ? kernel_of<64, true>(f) : kernel_of<128, true>(f);
+  return g == 0 ? kernel_of<32, false>(f) : g == 1 ? kernel_of<64, false>(f) : kernel_of<128, false>(f);
 }
 
-KernelFn kernel_for(int32_t group_size, uint32_t format) {
+KernelFn kernel_for(int32_t group_size, uint32_t format, bool y) {
   const int gi = group_size == 32 ? 0 : group_size == 64 ? 1 : 2;
-  return kernel_at(gi * kFormats + static_cast<int>(format & (kFormats - 1)));
+  return kernel_at((y ? 3 * kFormats : 0) + gi * kFormats + static_cast<int>(format & (kFormats - 1)));
 }
 
 bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE; }
@@ -157,6 +160,7 @@ struct Arrays {
   void* gis; int64_t ld_gis;
   void* yqt; int64_t ld_yqt;
   void* yst; int64_t ld_yst;
+  void* y = nullptr; int64_t ld_y = 0;   // optional bf16 y
 };
 
 // Contiguous arrays of the page's layout: x = [gate | up] [M, 2K], grad_y
@@ -207,6 +211,8 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   p.ld_giq = static_cast<int32_t>(a.ld_giq);
   p.ld_gis = static_cast<int32_t>(a.ld_gis);
   p.ld_yqt = a.ld_yqt;
+  p.y = static_cast<uint8_t*>(a.y);
+  p.ld_y = a.ld_y;
   p.ld_yst = a.ld_yst;
   p.num_tiles = p.Mg * p.Kg;
   p.yqt_vec16 = (a.ld_yqt % 16 == 0) ? 1 : 0;
@@ -226,7 +232,7 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format), mgate, mup, mdy, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format, a.y != nullptr), mgate, mup, mdy, p);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -291,7 +297,8 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
                          const void* grad_y, int64_t ld_grad_y, const void* grad_input_q,
                          int64_t ld_grad_input_q, const void* grad_input_s, int64_t ld_grad_input_s,
                          const void* y_q_t, int64_t ld_y_q_t, const void* y_s_t, int64_t ld_y_s_t,
-                         int64_t M, int64_t K, int32_t group_size, uint32_t format) {
+                         const void* y, int64_t ld_y, int64_t M, int64_t K, int32_t group_size,
+                         uint32_t format) {
   if (format & ~static_cast<uint32_t>(SDQ_FMT_E4M3 | SDQ_FMT_E8M0 | SDQ_FMT_YS_MG_K))
     return SDQ_ERR_FORMAT;
   if (!group_size_supported(group_size)) return SDQ_ERR_GROUP;
@@ -317,6 +324,10 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
   // rows of the bf16 inputs start on 16 bytes (tensor-map strides), rows of
   // grad_input_q on 16 bytes (vector stores)
   if ((ld_gate | ld_up | ld_grad_y) & 7 || ld_grad_input_q & 15) return SDQ_ERR_ALIGN;
+  if (y) {   // optional bf16 y: rows on 16 bytes
+    if (ld_y < K || ld_y > SDQ_MAX_LD) return SDQ_ERR_STRIDE;
+    if ((reinterpret_cast<uintptr_t>(y) & 15u) || (ld_y & 7)) return SDQ_ERR_ALIGN;
+  }
   return SDQ_OK;
 }
 
@@ -326,7 +337,8 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
   const Arrays a = packed(x, grad_y, const_cast<void*>(grad_input_q), const_cast<void*>(grad_input_s),
                           const_cast<void*>(y_q_t), const_cast<void*>(y_s_t), M, K, group_size, format);
   return sdq_validate_strided(a.gate, a.ld_gate, a.up, a.ld_up, a.gy, a.ld_gy, a.giq, a.ld_giq, a.gis,
-                              a.ld_gis, a.yqt, a.ld_yqt, a.yst, a.ld_yst, M, K, group_size, format);
+                              a.ld_gis, a.yqt, a.ld_yqt, a.yst, a.ld_yst, nullptr, 0, M, K, group_size,
+                              format);
 }
 
 int sdq_validate(const void* x, const void* grad_y, const int8_t* grad_input_q,
@@ -348,14 +360,15 @@ int sdq_fuse_format(const void* x, const void* grad_y, void* grad_input_q, void*
 int sdq_fuse_strided(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
                      const void* grad_y, int64_t ld_grad_y, void* grad_input_q,
                      int64_t ld_grad_input_q, void* grad_input_s, int64_t ld_grad_input_s,
-                     void* y_q_t, int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t, int64_t M,
-                     int64_t K, int32_t group_size, uint32_t format, void* stream) {
+                     void* y_q_t, int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t, void* y,
+                     int64_t ld_y, int64_t M, int64_t K, int32_t group_size, uint32_t format,
+                     void* stream) {
   const int st = sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q,
                                       ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t,
-                                      y_s_t, ld_y_s_t, M, K, group_size, format);
+                                      y_s_t, ld_y_s_t, y, ld_y, M, K, group_size, format);
   if (st != SDQ_OK || M == 0) return st;
   const Arrays a = {gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q, ld_grad_input_q,
-                    grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t};
+                    grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y};
   return launch(a, M, K, group_size, format, static_cast<cudaStream_t>(stream));
 }
 

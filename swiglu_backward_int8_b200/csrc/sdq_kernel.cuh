@@ -86,6 +86,8 @@ struct Params {
   int32_t K;
   int32_t Kg;        // 128-channel tiles per row
   int32_t gis_cols;  // 2K / group size: columns of grad_input_s (d_up groups from gis_cols/2)
+  uint8_t* y;        // optional bf16 y [M, K] (kernels built with kY)
+  int64_t ld_y;
   int64_t ld_yqt;    // elements from one row of each output to the next
   int64_t ld_yst;
   int32_t ld_giq;    // (at most 2^24: a tile's row offsets stay 32-bit products)
@@ -415,7 +417,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   }
 }
 
-template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK>
+template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK, bool kY>
 __global__ void __launch_bounds__(kThreads, 1)
     fuse_kernel(const __grid_constant__ CUtensorMap map_gate, const __grid_constant__ CUtensorMap map_up,
                 const __grid_constant__ CUtensorMap map_gy,
@@ -553,6 +555,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* yrow = yt + tok * (kG * 2);
         *reinterpret_cast<uint4*>(yrow + (ca ^ key) * 16) = make_uint4(yv[0], yv[1], yv[2], yv[3]);
         *reinterpret_cast<uint4*>(yrow + (cb ^ key) * 16) = make_uint4(yv[4], yv[5], yv[6], yv[7]);
+      }
+      if constexpr (kY) {   // y itself, bf16 (optional output): 16 bytes per chunk
+        const int yr = sub * kStageRows + srow;
+        if (yr < valid) {
+          int8_t* yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + yr) * p.ld_y + int64_t(j) * kG);
+          st_cs_v4(yg + ca * 16, make_uint4(yv[0], yv[1], yv[2], yv[3]));
+          st_cs_v4(yg + cb * 16, make_uint4(yv[4], yv[5], yv[6], yv[7]));
+        }
       }
 
       // ---- row amax of d_gate (hi half) and d_up (lo half) over the 8 lanes of the row

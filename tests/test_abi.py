@@ -165,7 +165,8 @@ def _strided_args(**kw):
     M, K = 256, 256
     a = dict(gate=A, ld_gate=2 * K, up=A + 2 * K, ld_up=2 * K, grad_y=A, ld_grad_y=K,
              grad_input_q=A, ld_grad_input_q=2 * K, grad_input_s=A, ld_grad_input_s=4,
-             y_q_t=A, ld_y_q_t=M, y_s_t=A, ld_y_s_t=2, M=M, K=K, group_size=128, format=0)
+             y_q_t=A, ld_y_q_t=M, y_s_t=A, ld_y_s_t=2, y=None, ld_y=0, M=M, K=K, group_size=128,
+             format=0)
     a.update(kw)
     return a
 
@@ -191,6 +192,13 @@ def _strided_args(**kw):
     (dict(group_size=64, ld_grad_input_s=7), 10),
     (dict(M=0, gate=0, up=0), 0),
     (dict(up=0), 1),
+    (dict(y=A, ld_y=256), 0),                            # the optional bf16 y
+    (dict(y=A, ld_y=264), 0),
+    (dict(y=A, ld_y=255), 10),                           # shorter than a row
+    (dict(y=A, ld_y=(1 << 36) + 8), 10),                 # above SDQ_MAX_LD
+    (dict(y=A, ld_y=260), 4),                            # rows must start on 16 bytes
+    (dict(y=A + 8, ld_y=256), 4),
+    (dict(y=None, ld_y=3), 0),                           # no y: its ld is not looked at
 ])
 def test_validate_strided_statuses(kw, status):
     import swiglu_backward_int8_b200 as sdq

@@ -22,9 +22,13 @@ def _padded(rows, cols, ld, dtype, fill):
     return buf, buf[:, :cols]
 
 
-def _run_strided(x_u16, gy_u16, G, fmt, pad, split):
+Y_SENTINEL = 0x7FC1   # a bf16 NaN the op never writes
+
+
+def _run_strided(x_u16, gy_u16, G, fmt, pad, split, with_y=False):
     """Run sdq_fuse_strided with every array padded by `pad` (elements);
-    returns numpy outputs like the format oracle, after checking the pads."""
+    returns numpy outputs like the format oracle (and, with_y, the optional
+    bf16 y as a fifth array), after checking the pads."""
     import swiglu_backward_int8_b200 as sdq
     codes, scales, layout = fmt
     M, K = gy_u16.shape
@@ -52,9 +56,13 @@ def _run_strided(x_u16, gy_u16, G, fmt, pad, split):
     yq = _padded(K, M, M + 13 * pad, torch.uint8, sq)     # often not a multiple of 16: byte stores
     ys = _padded(ys_shape[0], ys_shape[1], ys_shape[1] + pad, sdt, sfill)
     bits = (sdq.FMT_E4M3 if codes else 0) | (sdq.FMT_E8M0 if scales else 0) | (sdq.FMT_YS_MG_K if layout else 0)
+    yo = None
+    if with_y:   # bf16 y rows padded by 8 * pad elements, filled with a NaN sentinel
+        yo = _padded(M, K, K + bf_pad, torch.int16, Y_SENTINEL)
     sdq.sdq_fuse_strided(g_ptr, ld_g, u_ptr, ld_u, gyv.data_ptr(), ybuf.stride(0),
                          q[1].data_ptr(), q[0].stride(0), s[1].data_ptr(), s[0].stride(0),
                          yq[1].data_ptr(), yq[0].stride(0), ys[1].data_ptr(), ys[0].stride(0),
+                         yo[1].data_ptr() if with_y else None, yo[0].stride(0) if with_y else 0,
                          M, K, G, bits, torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert sdq.sdq_device_status() == 0
@@ -68,6 +76,10 @@ def _run_strided(x_u16, gy_u16, G, fmt, pad, split):
             want = sq if name in ("grad_input_q", "y_q_t") else U.SENTINEL_E8M0
             assert (pad_region == want).all(), f"{name}: padding written"
         out.append(view.cpu().numpy())
+    if with_y:
+        buf = yo[0].cpu().numpy().view(np.uint16)
+        assert (buf[:, K:] == Y_SENTINEL).all(), "y: padding written"
+        out.append(buf[:, :K].copy())
     return tuple(out)
 
 
@@ -117,3 +129,43 @@ def test_torch_views_of_wider_buffers():
     sdq.silu_dot_fwd_bwd_quant_fuse_split(xd[:, :256].clone(), xd[:, 256:].clone(), gyd, *outs2)
     for a, b in zip(outs2, ref):
         assert torch.equal(a.cpu(), b)
+
+
+@pytest.mark.parametrize("G,fmt", [(128, (0, 0, 0)), (64, (1, 1, 1)), (32, (0, 1, 0))])
+@pytest.mark.parametrize("M,K,split", [(1000, 256, False), (129, 384, True), (4096, 1408, False)])
+def test_optional_y_output(M, K, G, fmt, split):
+    """The optional bf16 y: within one bf16 step of the oracle's first-stage y
+    (the values y_q_t quantizes), padding untouched, and the four quantized
+    outputs bit-identical to the same call without it."""
+    w = W.small_workload(M, K, seed=M + 3 * K + G) if M != 4096 else W.WORKLOADS[1]
+    x, gy = W.make_inputs(w)
+    with_y = _run_strided(x, gy, G, fmt, pad=2, split=split, with_y=True)
+    without = _run_strided(x, gy, G, fmt, pad=2, split=split)
+    for a, b in zip(with_y[:4], without):
+        assert np.array_equal(a, b, equal_nan=True)
+    U.compare_bf16(with_y[4], oracle.swiglu_bwd_bf16(x, gy)[0], "y", f"M={M} K={K} G={G}")
+
+
+def test_optional_y_through_the_wrapper():
+    """``y=`` on the Python op (packed and split forms, y a view into a wider
+    buffer) gives the same y as the raw entry point and leaves the rest alone."""
+    import swiglu_backward_int8_b200 as sdq
+    w = W.small_workload(300, 256, seed=31)
+    x, gy = W.make_inputs(w)
+    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
+    ref = [t.cpu() for t in sdq.run(xd, gyd)]
+    raw = _run_strided(x, gy, 128, (0, 0, 0), pad=1, split=False, with_y=True)[4]
+    ybuf = torch.zeros(300, 256 + 8, dtype=torch.bfloat16, device="cuda")
+    outs = sdq.allocate_outputs(300, 256, "cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *outs, y=ybuf[:, :256])
+    for a, b in zip(outs, ref):
+        assert torch.equal(a.cpu(), b)
+    got = ybuf[:, :256].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, raw)
+    assert (ybuf[:, 256:] == 0).all()
+    y2 = torch.empty(300, 256, dtype=torch.bfloat16, device="cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse_split(xd[:, :256].clone(), xd[:, 256:].clone(), gyd,
+                                          *sdq.allocate_outputs(300, 256, "cuda"), y=y2)
+    assert np.array_equal(y2.cpu().view(torch.int16).numpy().view(np.uint16), raw)
+    with pytest.raises(ValueError):   # y must be bf16 [M, K]
+        sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *outs, y=torch.empty(300, 256, device="cuda"))
