@@ -73,6 +73,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.argtypes = [P, P, P, P, P, P, i64, i64, i64,
                                                              ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.oracle_silu_dot_fwd_bwd_quant_fuse_fmt.restype = ctypes.c_int
+        L.oracle_swiglu_bwd_bf16_dy.argtypes = [P, P, i64, i64, P, P, P]
+        L.oracle_swiglu_bwd_bf16_dy.restype = None
+        L.oracle_dequant_grad_y.argtypes = [P, P, i64, i64, P]
+        L.oracle_dequant_grad_y.restype = None
+        L.oracle_silu_dot_fwd_bwd_quant_fuse_qgrad.argtypes = [P, P, P, P, P, P, P, i64, i64, i64,
+                                                               ctypes.c_int, ctypes.c_int,
+                                                               ctypes.c_int]
+        L.oracle_silu_dot_fwd_bwd_quant_fuse_qgrad.restype = ctypes.c_int
         L.oracle_fp16_rne.argtypes = [dbl]
         L.oracle_fp16_rne.restype = ctypes.c_uint16
         L.oracle_q8_1_block.argtypes = [P, P]
@@ -228,6 +236,58 @@ def silu_dot_fwd_bwd_quant_fuse_fmt(x: np.ndarray, grad_y: np.ndarray, group_siz
     if rc != 0:
         raise ValueError(f"oracle rejected M={M} K={K} group_size={G} format "
                          f"({codes}, {scales}, {ys_layout})")
+    return giq, gis, yqt, yst
+
+
+# ---- grad_y handed over already quantized ------------------------------------
+
+def dequant_grad_y(grad_y_q: np.ndarray, grad_y_s: np.ndarray) -> np.ndarray:
+    """dy = q * s as float64 [M, K]: codes int8 [M, K], scales float32
+    [M, K/128], one per token and 128 consecutive channels."""
+    q = np.ascontiguousarray(grad_y_q, dtype=np.int8)
+    sc = np.ascontiguousarray(grad_y_s, dtype=np.float32)
+    M, K = q.shape
+    assert K % 128 == 0 and sc.shape == (M, K // 128), (q.shape, sc.shape)
+    dy = np.empty((M, K), np.float64)
+    lib().oracle_dequant_grad_y(_ptr(q), _ptr(sc), M, K, _ptr(dy))
+    return dy
+
+
+def swiglu_bwd_bf16_dy(x: np.ndarray, dy: np.ndarray):
+    """First stage on an fp64 grad_y: bf16 bit arrays (y, d_gate, d_up)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    M, K = dy.shape
+    assert x.shape == (M, 2 * K)
+    y = np.empty((M, K), np.uint16)
+    dg = np.empty((M, K), np.uint16)
+    du = np.empty((M, K), np.uint16)
+    lib().oracle_swiglu_bwd_bf16_dy(_ptr(x), _ptr(dy), M, K, _ptr(y), _ptr(dg), _ptr(du))
+    return y, dg, du
+
+
+def silu_dot_fwd_bwd_quant_fuse_qgrad(x: np.ndarray, grad_y_q: np.ndarray, grad_y_s: np.ndarray,
+                                      group_size: int = 128, codes: int = 0, scales: int = 0,
+                                      ys_layout: int = 0):
+    """The whole op with grad_y given quantized (INT8 codes [M, K], fp32
+    scales [M, K/128]); outputs as silu_dot_fwd_bwd_quant_fuse_fmt."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    q = np.ascontiguousarray(grad_y_q, dtype=np.int8)
+    sc = np.ascontiguousarray(grad_y_s, dtype=np.float32)
+    M, K = q.shape
+    assert x.shape == (M, 2 * K) and sc.shape == (M, K // 128), (x.shape, q.shape, sc.shape)
+    G = int(group_size)
+    sq, ss, yq, ys = output_shapes_fmt(M, K, G, ys_layout)
+    sdt = np.uint8 if scales else np.float32
+    giq = np.zeros(sq, np.uint8)
+    gis = np.zeros(ss, sdt)
+    yqt = np.zeros(yq, np.uint8)
+    yst = np.zeros(ys, sdt)
+    rc = lib().oracle_silu_dot_fwd_bwd_quant_fuse_qgrad(_ptr(x), _ptr(q), _ptr(sc), _ptr(giq),
+                                                        _ptr(gis), _ptr(yqt), _ptr(yst), M, K, G,
+                                                        int(codes), int(scales), int(ys_layout))
+    if rc != 0:
+        raise ValueError(f"oracle rejected M={M} K={K} group_size={G}")
     return giq, gis, yqt, yst
 
 

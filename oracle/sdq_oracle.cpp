@@ -70,6 +70,14 @@
 // nearest-even; an all-zero block has d = sum = 0 and q = 0; the block is
 // half2 (d, sum) first, then the 32 codes.  Pins: tests/test_oracle_fwd.py.
 //
+// A quantized grad_y (oracle_dequant_grad_y, oracle_swiglu_bwd_bf16_dy,
+// oracle_silu_dot_fwd_bwd_quant_fuse_qgrad; the reading is stated above
+// them).  Pins (tests/test_oracle_qgrad.py): with power-of-two scales every
+// q * s is a bf16 value, so the whole op must equal the pinned bf16-grad_y op
+// on that bf16 grad_y bit for bit; with any scales the first stage must equal
+// torch's float64 autograd of sum(q*s * silu(g) * u) rounded by the pinned
+// bf16 rounding.
+//
 // Pins (tests/test_oracle_formats.py): oracle_e4m3_rne against torch's
 // float8_e4m3fn conversion inside the finite range and against brute force
 // over all 127 finite magnitudes with exact rationals; oracle_e8m0_ceil
@@ -168,23 +176,30 @@ void oracle_quant_group(const uint16_t* v, int64_t n, int64_t stride,
   *scale = s;
 }
 
-// First stage: the bf16 values y, d_gate, d_up ([M, K] each, bf16 bits) from
-// x = [gate | up] ([M, 2K]) and grad_y ([M, K]).
-void oracle_swiglu_bwd_bf16(const uint16_t* x, const uint16_t* grad_y,
-                            int64_t M, int64_t K, uint16_t* y,
-                            uint16_t* d_gate, uint16_t* d_up) {
+// First stage on grad_y given as fp64 values dy [M, K]: the bf16 values y,
+// d_gate, d_up ([M, K] each, bf16 bits) from x = [gate | up] ([M, 2K]).
+void oracle_swiglu_bwd_bf16_dy(const uint16_t* x, const double* dy, int64_t M, int64_t K,
+                               uint16_t* y, uint16_t* d_gate, uint16_t* d_up) {
   for (int64_t m = 0; m < M; ++m) {
     for (int64_t k = 0; k < K; ++k) {
       const double g = bf16_to_float(x[m * 2 * K + k]);
       const double u = bf16_to_float(x[m * 2 * K + K + k]);
-      const double dy = bf16_to_float(grad_y[m * K + k]);
       double yv, dg, du;
-      oracle_swiglu_bwd_fp64(g, u, dy, &yv, &dg, &du);
+      oracle_swiglu_bwd_fp64(g, u, dy[m * K + k], &yv, &dg, &du);
       y[m * K + k] = oracle_bf16_rne(yv);
       d_gate[m * K + k] = oracle_bf16_rne(dg);
       d_up[m * K + k] = oracle_bf16_rne(du);
     }
   }
+}
+
+// First stage on a bf16 grad_y ([M, K] bf16 bits): its exact values.
+void oracle_swiglu_bwd_bf16(const uint16_t* x, const uint16_t* grad_y,
+                            int64_t M, int64_t K, uint16_t* y,
+                            uint16_t* d_gate, uint16_t* d_up) {
+  std::vector<double> dy(M * K);
+  for (int64_t i = 0; i < M * K; ++i) dy[i] = bf16_to_float(grad_y[i]);
+  oracle_swiglu_bwd_bf16_dy(x, dy.data(), M, K, y, d_gate, d_up);
 }
 
 // The whole op.  Returns 0, or -1 for arguments the definition does not cover
@@ -310,6 +325,11 @@ void oracle_quant_group_fmt(const uint16_t* v, int64_t n, int64_t stride, uint8_
 // The whole op in a chosen format.  codes / scales as in
 // oracle_quant_group_fmt; ys_layout: 0 y_s_t [K, Mg], 1 [Mg, K].  Code
 // arrays are bytes; scale arrays are fp32 or one byte per scale.
+static void quantize_outputs_fmt(const uint16_t* y, const uint16_t* dg, const uint16_t* du,
+                                 uint8_t* grad_input_q, void* grad_input_s, uint8_t* y_q_t,
+                                 void* y_s_t, int64_t M, int64_t K, int64_t G, int codes,
+                                 int scales, int ys_layout);
+
 int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* grad_y,
                                            uint8_t* grad_input_q, void* grad_input_s,
                                            uint8_t* y_q_t, void* y_s_t, int64_t M, int64_t K,
@@ -319,13 +339,58 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
   if (G < 1 || M < 0 || K < 0 || K % G != 0) return -1;
   if (codes < 0 || codes > 1 || scales < 0 || scales > 1 || ys_layout < 0 || ys_layout > 1) return -1;
   if (M == 0 || K == 0) return 0;
+  std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
+  oracle_swiglu_bwd_bf16(x, grad_y, M, K, y.data(), dg.data(), du.data());
+  quantize_outputs_fmt(y.data(), dg.data(), du.data(), grad_input_q, grad_input_s, y_q_t, y_s_t,
+                       M, K, G, codes, scales, ys_layout);
+  return 0;
+}
+
+// ---- grad_y handed over already quantized (the chained backward) -------------
+//
+// Reading: the upstream step hands grad_y over in the row-group format this
+// op itself writes for grad_input: INT8 codes q [M, K] and fp32 scales
+// s [M, K/128], one per token and 128 consecutive channels; the value it
+// stands for is q * s (exact in fp64: 8 x 24 significant bits).
+
+// dy[m, k] = q[m, k] * s[m, k / 128].
+void oracle_dequant_grad_y(const int8_t* q, const float* s, int64_t M, int64_t K, double* dy) {
+  const int64_t Kg = K / 128;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k)
+      dy[m * K + k] = static_cast<double>(q[m * K + k]) * static_cast<double>(s[m * Kg + k / 128]);
+}
+
+// The whole op with a quantized grad_y (K a multiple of 128), outputs as in
+// oracle_silu_dot_fwd_bwd_quant_fuse_fmt.
+int oracle_silu_dot_fwd_bwd_quant_fuse_qgrad(const uint16_t* x, const int8_t* grad_y_q,
+                                             const float* grad_y_s, uint8_t* grad_input_q,
+                                             void* grad_input_s, uint8_t* y_q_t, void* y_s_t,
+                                             int64_t M, int64_t K, int64_t group_size, int codes,
+                                             int scales, int ys_layout) {
+  const int64_t G = group_size;
+  if (G < 1 || M < 0 || K < 0 || K % G != 0 || K % 128 != 0) return -1;
+  if (codes < 0 || codes > 1 || scales < 0 || scales > 1 || ys_layout < 0 || ys_layout > 1) return -1;
+  if (M == 0 || K == 0) return 0;
+  std::vector<double> dy(M * K);
+  oracle_dequant_grad_y(grad_y_q, grad_y_s, M, K, dy.data());
+  std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
+  oracle_swiglu_bwd_bf16_dy(x, dy.data(), M, K, y.data(), dg.data(), du.data());
+  quantize_outputs_fmt(y.data(), dg.data(), du.data(), grad_input_q, grad_input_s, y_q_t, y_s_t,
+                       M, K, G, codes, scales, ys_layout);
+  return 0;
+}
+
+// The two quantizations of the first stage's bf16 y, d_gate, d_up.
+static void quantize_outputs_fmt(const uint16_t* y, const uint16_t* dg, const uint16_t* du,
+                                 uint8_t* grad_input_q, void* grad_input_s, uint8_t* y_q_t,
+                                 void* y_s_t, int64_t M, int64_t K, int64_t G, int codes,
+                                 int scales, int ys_layout) {
   const int64_t Kg = K / G;
   const int64_t Mg = (M + G - 1) / G;
   const int64_t sb = scales ? 1 : 4;   // bytes per scale
   uint8_t* gis = static_cast<uint8_t*>(grad_input_s);
   uint8_t* yst = static_cast<uint8_t*>(y_s_t);
-  std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
-  oracle_swiglu_bwd_bf16(x, grad_y, M, K, y.data(), dg.data(), du.data());
   for (int64_t m = 0; m < M; ++m) {
     for (int64_t j = 0; j < 2 * Kg; ++j) {
       const uint16_t* src = (j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G];
@@ -342,7 +407,6 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
                              scales);
     }
   }
-  return 0;
 }
 
 // ---- forward-side neighbour: SwiGLU forward + q8_1 rows -----------------------

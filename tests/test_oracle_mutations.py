@@ -69,10 +69,20 @@ MUTATIONS = [
      "test_swiglu_rows_blocks_are_the_rows_32_value_blocks", "fwd"),
     ("if (limit > 0.0) {   // false for NaN: no clamp", "if (limit != 0.0) {",
      "test_swiglu_rows_closed_form_without_clamp", "fwd"),
+    # a quantized grad_y (pins in test_oracle_qgrad.py)
+    ("static_cast<double>(s[m * Kg + k / 128])", "static_cast<double>(s[m * Kg + k % Kg])",
+     "test_whole_op_pow2_scales_equals_bf16_op", "qgrad"),
+    ("static_cast<double>(s[m * Kg + k / 128])", "static_cast<double>(s[(k / 128) * M + m])",
+     "test_whole_op_pow2_scales_equals_bf16_op", "qgrad"),
+    ("static_cast<double>(q[m * K + k])", "static_cast<double>(static_cast<uint8_t>(q[m * K + k]))",
+     "test_first_stage_against_autograd", "qgrad"),
+    ("static_cast<double>(q[m * K + k]) * static_cast<double>(s[m * Kg + k / 128])",
+     "static_cast<double>(static_cast<float>(q[m * K + k]) * s[m * Kg + k / 128])",
+     "test_dequant_is_exact_in_fp64", "qgrad"),
 ]
 
 PIN_FILES = {"pins": "test_oracle_pins.py", "formats": "test_oracle_formats.py",
-             "fwd": "test_oracle_fwd.py"}
+             "fwd": "test_oracle_fwd.py", "qgrad": "test_oracle_qgrad.py"}
 
 
 def _run_mutant(tmp_dir, idx, old, new, pin, pins="pins"):
