@@ -77,6 +77,8 @@ def parse_args():
                     help="fuse: the backward op (the headline); swiglu_q8_1: the forward-side "
                          "SwiGLU + q8_1 rows on the workload's gate and up (rows = M, inter = K)")
     ap.add_argument("--limit", type=float, default=0.0, help="swiglu_q8_1: the clamp (0: none)")
+    ap.add_argument("--int8-grad-y", action="store_true",
+                    help="also time the call with grad_y given as INT8 codes + fp32 scales")
     ap.add_argument("--with-y", action="store_true",
                     help="also time the call with the optional bf16 y output")
     ap.add_argument("--all-formats", action="store_true",
@@ -285,8 +287,14 @@ def scale_bytes(fmt) -> int:
     return 1 if fmt[1] == "e8m0" else 4
 
 
+def int8_grad_y_bytes(w: W.Workload) -> int:
+    """Algorithmic bytes of one call with grad_y as INT8 codes + fp32 scales."""
+    return w.algorithmic_bytes() - 2 * w.M * w.K + w.M * w.K + 4 * w.M * (w.K // 128)
+
+
 def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, fmt=PAGE_FORMAT,
-                   with_y: bool = False):
+                   with_y: bool = False, int8_grad_y=None):
+    """int8_grad_y: None, or (codes, scales) numpy arrays used in place of gy_np."""
     import torch
     import swiglu_backward_int8_b200 as sdq
     M, K = w.M, w.K
@@ -294,20 +302,26 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
     footprint = w.algorithmic_bytes(scale_bytes(fmt)) + (2 * M * K if with_y else 0)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nsets = max(1, -(-3 * l2 // footprint))
-    x0, g0 = _to_device_bf16(x_np, device), _to_device_bf16(gy_np, device)
+    x0 = _to_device_bf16(x_np, device)
+    if int8_grad_y is None:
+        g0, gs0 = _to_device_bf16(gy_np, device), None
+    else:
+        g0 = torch.from_numpy(int8_grad_y[0]).to(device)
+        gs0 = torch.from_numpy(int8_grad_y[1]).to(device)
     sets = []
     for s in range(nsets):
         xs = x0 if s == 0 else x0.clone()
         gs = g0 if s == 0 else g0.clone()
-        sets.append((xs, gs, sdq.allocate_outputs(M, K, device, codes=codes, scales=scales,
-                                                  y_scale_layout=layout),
+        gss = gs0 if (s == 0 or gs0 is None) else gs0.clone()
+        sets.append((xs, gs, gss, sdq.allocate_outputs(M, K, device, codes=codes, scales=scales,
+                                                       y_scale_layout=layout),
                      torch.empty(M, K, dtype=torch.bfloat16, device=device) if with_y else None))
     stream = torch.cuda.current_stream(device)
 
     def call(k):
-        xs, gs, outs, ys = sets[k % nsets]
+        xs, gs, gss, outs, ys = sets[k % nsets]
         sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, codes=codes, scales=scales,
-                                        y_scale_layout=layout, y=ys)
+                                        y_scale_layout=layout, y=ys, grad_y_s=gss)
 
     for k in range(warmup):
         call(k)
@@ -452,6 +466,18 @@ def run_sdq(args):
         with_y = {"us_per_call": us, "GB_s": gbs, "frac_of_measured_hbm": gbs / peak,
                   "algorithmic_bytes_per_launch": yb, "format": format_name(PAGE_FORMAT)}
 
+    int8_gy = None
+    if args.int8_grad_y:   # grad_y handed over as INT8 codes + fp32 scales
+        qgy = W.quantized_grad_y(wr)
+        qms, _, _ = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device,
+                                   int8_grad_y=qgy)
+        qms = parallel.max_over_ranks(qms, device)
+        us = qms / args.steps * 1e3
+        qb = int8_grad_y_bytes(w)
+        gbs = qb / (us * 1e-6) / 1e9
+        int8_gy = {"us_per_call": us, "GB_s": gbs, "frac_of_measured_hbm": gbs / peak,
+                   "algorithmic_bytes_per_launch": qb, "format": format_name(PAGE_FORMAT)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0)
@@ -482,6 +508,8 @@ def run_sdq(args):
             line["per_format"] = per_fmt
         if with_y is not None:
             line["with_y"] = with_y
+        if int8_gy is not None:
+            line["int8_grad_y"] = int8_gy
         print(json.dumps(line), flush=True)
     import torch.distributed as tdist
     if tdist.is_initialized():

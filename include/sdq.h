@@ -198,6 +198,36 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
                          int64_t M, int64_t K, int32_t group_size, uint32_t format);
 
 /*
+ * sdq_fuse_int8_grad_y -- sdq_fuse_strided with grad_y handed over already
+ * quantized, as the step after the op in a chained INT8 backward would hand
+ * it over: in the row-group format this op writes for grad_input.  The page
+ * ("entry point" section) takes grad_y in bf16; this entry reads
+ *   grad_y_q   device, INT8 codes [M, K]; 16-byte aligned; ld a multiple of
+ *              16 (rows start on 16 bytes), K <= ld <= SDQ_MAX_LD
+ *   grad_y_s   device, fp32 scales [M, K/128], one per token and 128
+ *              consecutive channels; 4-byte aligned; K/128 <= ld <= SDQ_MAX_LD
+ * and takes grad_y[m, k] = grad_y_q[m, k] * grad_y_s[m, k / 128], each
+ * product rounded once to fp32; everything else (the optional y included)
+ * as sdq_fuse_strided.  Statuses as sdq_fuse_strided, plus SDQ_ERR_NULL for a
+ * NULL grad_y_s.
+ */
+int sdq_fuse_int8_grad_y(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                         const void* grad_y_q, int64_t ld_grad_y_q, const float* grad_y_s,
+                         int64_t ld_grad_y_s, void* grad_input_q, int64_t ld_grad_input_q,
+                         void* grad_input_s, int64_t ld_grad_input_s, void* y_q_t,
+                         int64_t ld_y_q_t, void* y_s_t, int64_t ld_y_s_t, void* y, int64_t ld_y,
+                         int64_t M, int64_t K, int32_t group_size, uint32_t format, void* stream);
+
+/* The argument checks of sdq_fuse_int8_grad_y alone: no CUDA call, no launch. */
+int sdq_validate_int8_grad_y(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                             const void* grad_y_q, int64_t ld_grad_y_q, const float* grad_y_s,
+                             int64_t ld_grad_y_s, const void* grad_input_q,
+                             int64_t ld_grad_input_q, const void* grad_input_s,
+                             int64_t ld_grad_input_s, const void* y_q_t, int64_t ld_y_q_t,
+                             const void* y_s_t, int64_t ld_y_s_t, const void* y, int64_t ld_y,
+                             int64_t M, int64_t K, int32_t group_size, uint32_t format);
+
+/*
  * sdq_swiglu_q8_1 -- the forward-side neighbour of the backward op: the
  * SwiGLU forward and the q8_1 row quantization of its output in one pass.
  * Source: the launcher kquant_swiglu_q8_1_rows on the page with the K-quant

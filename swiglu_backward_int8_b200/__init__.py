@@ -23,13 +23,15 @@ import torch
 
 from ._lib import (FMT_E4M3, FMT_E8M0, FMT_YS_MG_K, LIB_PATH, SdqError, Status, last_cuda_error,
                    sdq_device_status, sdq_fuse, sdq_fuse_format, sdq_fuse_host,
-                   sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_fuse_strided,
+                   sdq_fuse_host_noalloc, sdq_fuse_host_workspace_bytes, sdq_fuse_int8_grad_y,
+                   sdq_fuse_strided, sdq_validate_int8_grad_y,
                    sdq_swiglu_q8_1, sdq_validate, sdq_validate_format, sdq_validate_strided,
                    sdq_validate_swiglu_q8_1, status_string, version)
 
 __all__ = [
     "silu_dot_fwd_bwd_quant_fuse", "silu_dot_fwd_bwd_quant_fuse_split",
     "silu_dot_fwd_bwd_quant_fuse_host", "allocate_outputs", "sdq_fuse_strided", "sdq_validate_strided",
+    "sdq_fuse_int8_grad_y", "sdq_validate_int8_grad_y",
     "swiglu_q8_1", "sdq_swiglu_q8_1", "sdq_validate_swiglu_q8_1", "Q8_1_BLOCK_BYTES",
     "output_shapes", "output_format", "sdq_fuse", "sdq_fuse_format", "sdq_validate_format",
     "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
@@ -121,7 +123,7 @@ def _check_outputs(M, K, outs, group_size, want_cuda, codes, scales, y_scale_lay
 
 
 def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", scales="fp32",
-                   y_scale_layout="k_mg"):
+                   y_scale_layout="k_mg", grad_y_s=None):
     if x.dim() != 2 or grad_y.dim() != 2:
         raise ValueError("x and grad_y must be 2-D")
     M, K2 = x.shape
@@ -131,9 +133,12 @@ def _check_tensors(x, grad_y, outs, group_size, want_cuda: bool, codes="int8", s
     _check_group(K, group_size, want_cuda)
     bf16 = (torch.bfloat16,)
     ld_x = _rows("x", x, (M, 2 * K), bf16, want_cuda, x.device)
-    ld_gy = _rows("grad_y", grad_y, (M, K), bf16, want_cuda, x.device)
+    if grad_y_s is None:
+        ld_gy, gys = _rows("grad_y", grad_y, (M, K), bf16, want_cuda, x.device), (None, 0)
+    else:
+        ld_gy, *gys = _grad_y(grad_y, grad_y_s, M, K, x.device)
     lds = _check_outputs(M, K, outs, group_size, want_cuda, codes, scales, y_scale_layout, x.device)
-    return M, K, ld_x, ld_gy, lds
+    return M, K, ld_x, ld_gy, lds, tuple(gys)
 
 
 def _check_y(y, M, K, device):
@@ -143,22 +148,39 @@ def _check_y(y, M, K, device):
     return y.data_ptr(), _rows("y", y, (M, K), (torch.bfloat16,), True, device)
 
 
+def _grad_y(grad_y, grad_y_s, M, K, device):
+    """grad_y in bf16 [M, K], or INT8 codes [M, K] with fp32 scales
+    ``grad_y_s`` [M, K/128]: (its leading dimension, the scales' pointer or
+    None, their leading dimension)."""
+    if grad_y_s is None:
+        return _rows("grad_y", grad_y, (M, K), (torch.bfloat16,), True, device), None, 0
+    ld_q = _rows("grad_y", grad_y, (M, K), (torch.int8,), True, device)
+    ld_s = _rows("grad_y_s", grad_y_s, (M, K // GROUP_SIZE), (torch.float32,), True, device)
+    return ld_q, grad_y_s.data_ptr(), ld_s
+
+
 def _call_strided(gate, ld_gate, up, ld_up, grad_y, ld_gy, outs, lds, M, K, group_size, fmt, device,
-                  y=None):
+                  y=None, gys=None, ld_gys=0):
     yp, ld_y = _check_y(y, M, K, device)
     with torch.cuda.device(device):
         stream = torch.cuda.current_stream(device).cuda_stream
         q, s, yq, ys = outs
-        sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y.data_ptr(), ld_gy, q.data_ptr(), lds[0],
-                         s.data_ptr(), lds[1], yq.data_ptr(), lds[2], ys.data_ptr(), lds[3], yp,
-                         ld_y, M, K, group_size, fmt, stream)
+        if gys is None:
+            sdq_fuse_strided(gate, ld_gate, up, ld_up, grad_y.data_ptr(), ld_gy, q.data_ptr(),
+                             lds[0], s.data_ptr(), lds[1], yq.data_ptr(), lds[2], ys.data_ptr(),
+                             lds[3], yp, ld_y, M, K, group_size, fmt, stream)
+        else:
+            sdq_fuse_int8_grad_y(gate, ld_gate, up, ld_up, grad_y.data_ptr(), ld_gy, gys, ld_gys,
+                                 q.data_ptr(), lds[0], s.data_ptr(), lds[1], yq.data_ptr(), lds[2],
+                                 ys.data_ptr(), lds[3], yp, ld_y, M, K, group_size, fmt, stream)
 
 
 def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_input_q: torch.Tensor,
                                 grad_input_s: torch.Tensor, y_q_t: torch.Tensor,
                                 y_s_t: torch.Tensor, group_size: int = GROUP_SIZE, *,
                                 codes: Optional[str] = None, scales: Optional[str] = None,
-                                y_scale_layout: str = "k_mg", y: Optional[torch.Tensor] = None) -> None:
+                                y_scale_layout: str = "k_mg", y: Optional[torch.Tensor] = None,
+                                grad_y_s: Optional[torch.Tensor] = None) -> None:
     """Fused SwiGLU backward + dual-axis quantization, in place, on the
     current CUDA stream of x's device.  The code format ("int8" or "e4m3")
     and the scale format ("fp32" or "e8m0") follow the dtypes of
@@ -166,16 +188,18 @@ def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_inpu
     (y_s_t [K, ceil(M/G)]) or "mg_k"; ``group_size`` is 128, 64 or 32.  Every
     tensor is 2-D row-major; rows may be padded (a slice of a wider buffer):
     the library takes each tensor's row stride.  ``y`` (bf16 [M, K], optional)
-    also receives the recomputed y itself, the values y_q_t quantizes.
+    also receives the recomputed y itself, the values y_q_t quantizes.  With
+    ``grad_y_s`` (fp32 [M, K/128]) grad_y is INT8 codes [M, K] standing for
+    grad_y * grad_y_s[m, k // 128] (grad_y handed over already quantized).
     Raises ValueError on bad arguments and SdqError on a library status."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
     codes = _infer("codes", codes, grad_input_q, _CODE_DTYPES)
     scales = _infer("scales", scales, grad_input_s, _SCALE_DTYPES)
     fmt = output_format(codes, scales, y_scale_layout)
-    M, K, ld_x, ld_gy, lds = _check_tensors(x, grad_y, outs, group_size, True, codes, scales,
-                                            y_scale_layout)
+    M, K, ld_x, ld_gy, lds, gys = _check_tensors(x, grad_y, outs, group_size, True, codes, scales,
+                                                 y_scale_layout, grad_y_s)
     _call_strided(x.data_ptr(), ld_x, x.data_ptr() + 2 * K, ld_x, grad_y, ld_gy, outs, lds, M, K,
-                  group_size, fmt, x.device, y)
+                  group_size, fmt, x.device, y, *gys)
 
 
 def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad_y: torch.Tensor,
@@ -184,7 +208,8 @@ def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad
                                       group_size: int = GROUP_SIZE, *, codes: Optional[str] = None,
                                       scales: Optional[str] = None,
                                       y_scale_layout: str = "k_mg",
-                                      y: Optional[torch.Tensor] = None) -> None:
+                                      y: Optional[torch.Tensor] = None,
+                                      grad_y_s: Optional[torch.Tensor] = None) -> None:
     """The op with gate and up as two [M, K] bf16 tensors instead of one
     x = [gate | up] (e.g. the two halves of a fused projection kept apart);
     otherwise as silu_dot_fwd_bwd_quant_fuse."""
@@ -199,10 +224,10 @@ def silu_dot_fwd_bwd_quant_fuse_split(gate: torch.Tensor, up: torch.Tensor, grad
     bf16 = (torch.bfloat16,)
     ld_g = _rows("gate", gate, (M, K), bf16, True, gate.device)
     ld_u = _rows("up", up, (M, K), bf16, True, gate.device)
-    ld_gy = _rows("grad_y", grad_y, (M, K), bf16, True, gate.device)
+    ld_gy, gys, ld_gys = _grad_y(grad_y, grad_y_s, M, K, gate.device)
     lds = _check_outputs(M, K, outs, group_size, True, codes, scales, y_scale_layout, gate.device)
     _call_strided(gate.data_ptr(), ld_g, up.data_ptr(), ld_u, grad_y, ld_gy, outs, lds, M, K,
-                  group_size, fmt, gate.device, y)
+                  group_size, fmt, gate.device, y, gys, ld_gys)
 
 
 def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
@@ -215,7 +240,7 @@ def silu_dot_fwd_bwd_quant_fuse_host(x: torch.Tensor, grad_y: torch.Tensor,
     device ``workspace`` (uint8 CUDA tensor of at least
     ``sdq_fuse_host_workspace_bytes(M, K, chunk_rows)`` bytes)."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)
-    M, K, _, _, _ = _check_tensors(x, grad_y, outs, group_size, want_cuda=False)
+    M, K, _, _, _, _ = _check_tensors(x, grad_y, outs, group_size, want_cuda=False)
     if not workspace.is_cuda:
         raise ValueError("workspace must be a CUDA tensor")
     dev = device or workspace.device

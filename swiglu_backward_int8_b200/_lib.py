@@ -37,6 +37,11 @@ _lib.sdq_fuse_strided.argtypes = _STRIDED + [_P]
 _lib.sdq_fuse_strided.restype = ctypes.c_int
 _lib.sdq_validate_strided.argtypes = _STRIDED
 _lib.sdq_validate_strided.restype = ctypes.c_int
+_INT8_GY = [_P, _I64] * 9 + [_I64, _I64, _I32, ctypes.c_uint32]
+_lib.sdq_fuse_int8_grad_y.argtypes = _INT8_GY + [_P]
+_lib.sdq_fuse_int8_grad_y.restype = ctypes.c_int
+_lib.sdq_validate_int8_grad_y.argtypes = _INT8_GY
+_lib.sdq_validate_int8_grad_y.restype = ctypes.c_int
 _lib.sdq_swiglu_q8_1.argtypes = [_P, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _I64, ctypes.c_float, _P]
 _lib.sdq_swiglu_q8_1.restype = ctypes.c_int
 _lib.sdq_validate_swiglu_q8_1.argtypes = [_P, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _I64]
@@ -146,6 +151,34 @@ def sdq_validate_strided(gate: int, ld_gate: int, up: int, ld_up: int, grad_y: i
                                          ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t,
                                          ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y, M, K, group_size,
                                          format))
+
+
+def sdq_fuse_int8_grad_y(gate: int, ld_gate: int, up: int, ld_up: int, grad_y_q: int,
+                         ld_grad_y_q: int, grad_y_s: int, ld_grad_y_s: int, grad_input_q: int,
+                         ld_grad_input_q: int, grad_input_s: int, ld_grad_input_s: int, y_q_t: int,
+                         ld_y_q_t: int, y_s_t: int, ld_y_s_t: int, y: Optional[int], ld_y: int,
+                         M: int, K: int, group_size: int = 128, format: int = 0,
+                         stream: Optional[int] = None) -> None:
+    """Raw-pointer form of the entry point taking grad_y as INT8 codes and
+    fp32 scales (leading dimensions in elements)."""
+    _check(_lib.sdq_fuse_int8_grad_y(gate, ld_gate, up, ld_up, grad_y_q, ld_grad_y_q, grad_y_s,
+                                     ld_grad_y_s, grad_input_q, ld_grad_input_q, grad_input_s,
+                                     ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y, M,
+                                     K, group_size, format, stream or 0),
+           "sdq_fuse_int8_grad_y")
+
+
+def sdq_validate_int8_grad_y(gate: int, ld_gate: int, up: int, ld_up: int, grad_y_q: int,
+                             ld_grad_y_q: int, grad_y_s: int, ld_grad_y_s: int, grad_input_q: int,
+                             ld_grad_input_q: int, grad_input_s: int, ld_grad_input_s: int,
+                             y_q_t: int, ld_y_q_t: int, y_s_t: int, ld_y_s_t: int,
+                             y: Optional[int], ld_y: int, M: int, K: int, group_size: int = 128,
+                             format: int = 0) -> int:
+    """Argument checks of sdq_fuse_int8_grad_y only (no CUDA call); returns the status code."""
+    return int(_lib.sdq_validate_int8_grad_y(gate, ld_gate, up, ld_up, grad_y_q, ld_grad_y_q,
+                                             grad_y_s, ld_grad_y_s, grad_input_q, ld_grad_input_q,
+                                             grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t,
+                                             ld_y_s_t, y, ld_y, M, K, group_size, format))
 
 
 def sdq_swiglu_q8_1(gate: int, ld_gate: int, up: int, ld_up: int, w: Optional[int], h: int, ld_h: int,

@@ -25,36 +25,48 @@ constexpr int kStages = SDQ_STAGES;
 constexpr int kMaxDevices = 64;
 
 // One kernel per group size (32, 64, 128), output format (SDQ_FMT_* bits
-// 0..2) and whether bf16 y is written too.
+// 0..2), whether bf16 y is written too, and whether grad_y comes as INT8
+// codes with scales.
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const sdq::Params);
 constexpr int kFormats = 8;
-constexpr int kKernels = 2 * 3 * kFormats;
+constexpr int kKernels = 2 * 2 * 3 * kFormats;
 
-template <int G, bool kY>
+template <int G, bool kY, bool kQ>
 constexpr KernelFn kernel_of(int f) {
   switch (f) {
-    case 0: return sdq::fuse_kernel<kStages, G, false, false, false, kY>;
-    case 1: return sdq::fuse_kernel<kStages, G, true, false, false, kY>;
-    case 2: return sdq::fuse_kernel<kStages, G, false, true, false, kY>;
-    case 3: return sdq::fuse_kernel<kStages, G, true, true, false, kY>;
-    case 4: return sdq::fuse_kernel<kStages, G, false, false, true, kY>;
-    case 5: return sdq::fuse_kernel<kStages, G, true, false, true, kY>;
-    case 6: return sdq::fuse_kernel<kStages, G, false, true, true, kY>;
-    default: return sdq::fuse_kernel<kStages, G, true, true, true, kY>;
+    case 0: return sdq::fuse_kernel<kStages, G, false, false, false, kY, kQ>;
+    case 1: return sdq::fuse_kernel<kStages, G, true, false, false, kY, kQ>;
+    case 2: return sdq::fuse_kernel<kStages, G, false, true, false, kY, kQ>;
+    case 3: return sdq::fuse_kernel<kStages, G, true, true, false, kY, kQ>;
+    case 4: return sdq::fuse_kernel<kStages, G, false, false, true, kY, kQ>;
+    case 5: return sdq::fuse_kernel<kStages, G, true, false, true, kY, kQ>;
+    case 6: return sdq::fuse_kernel<kStages, G, false, true, true, kY, kQ>;
+    default: return sdq::fuse_kernel<kStages, G, true, true, true, kY, kQ>;
   }
 }
 
-// Kernel number n = 24 * (y written) + 8 * (0, 1, 2 for group size 32, 64, 128) + format bits.
-KernelFn kernel_at(int n) {
-  const bool y = n >= 3 * kFormats;
-  const int g = (n % (3 * kFormats)) / kFormats, f = n % kFormats;
-  if (y) return g == 0 ? kernel_of<32, true>(f) : g == 1 ? kernel_of<64, true>(f) : kernel_of<128, true>(f);
-  return g == 0 ? kernel_of<32, false>(f) : g == 1 ? kernel_of<64, false>(f) : kernel_of<128, false>(f);
+template <bool kY, bool kQ>
+KernelFn kernel_of_group(int g, int f) {
+  return g == 0 ? kernel_of<32, kY, kQ>(f) : g == 1 ? kernel_of<64, kY, kQ>(f) : kernel_of<128, kY, kQ>(f);
 }
 
-KernelFn kernel_for(int32_t group_size, uint32_t format, bool y) {
+// Kernel number n = 48 * (INT8 grad_y) + 24 * (y written) + 8 * (0, 1, 2 for
+// group size 32, 64, 128) + format bits.
+KernelFn kernel_at(int n) {
+  const int v = n / (3 * kFormats);   // 0..3: (y, INT8 grad_y) bits
+  const int g = (n % (3 * kFormats)) / kFormats, f = n % kFormats;
+  switch (v) {
+    case 0: return kernel_of_group<false, false>(g, f);
+    case 1: return kernel_of_group<true, false>(g, f);
+    case 2: return kernel_of_group<false, true>(g, f);
+    default: return kernel_of_group<true, true>(g, f);
+  }
+}
+
+KernelFn kernel_for(int32_t group_size, uint32_t format, bool y, bool qdy) {
   const int gi = group_size == 32 ? 0 : group_size == 64 ? 1 : 2;
-  return kernel_at((y ? 3 * kFormats : 0) + gi * kFormats + static_cast<int>(format & (kFormats - 1)));
+  return kernel_at(((qdy ? 2 : 0) + (y ? 1 : 0)) * 3 * kFormats + gi * kFormats +
+                   static_cast<int>(format & (kFormats - 1)));
 }
 
 bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE; }
@@ -135,15 +147,18 @@ int current_device(DeviceState** out) {
   return SDQ_OK;
 }
 
+// A [rows, inner] row-major array of bf16 (or, with `bytes`, 8-bit codes)
+// read in boxes of 64 rows x 128 elements.
 int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-             uint64_t row_bytes) {
+             uint64_t row_bytes, bool bytes = false) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(sdq::kG), static_cast<cuuint32_t>(sdq::kStageRows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
@@ -161,6 +176,7 @@ struct Arrays {
   void* yqt; int64_t ld_yqt;
   void* yst; int64_t ld_yst;
   void* y = nullptr; int64_t ld_y = 0;   // optional bf16 y
+  const void* gys = nullptr; int64_t ld_gys = 0;   // set: gy holds INT8 codes, these their scales
 };
 
 // Contiguous arrays of the page's layout: x = [gate | up] [M, 2K], grad_y
@@ -197,7 +213,8 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   CUtensorMap mgate, mup, mdy;
   if ((st = make_map(&mgate, a.gate, K, M, 2 * a.ld_gate)) != SDQ_OK) return st;
   if ((st = make_map(&mup, a.up, K, M, 2 * a.ld_up)) != SDQ_OK) return st;
-  if ((st = make_map(&mdy, a.gy, K, M, 2 * a.ld_gy)) != SDQ_OK) return st;
+  const bool qdy = a.gys != nullptr;
+  if ((st = make_map(&mdy, a.gy, K, M, (qdy ? 1 : 2) * a.ld_gy, qdy)) != SDQ_OK) return st;
   sdq::Params p;
   p.giq = static_cast<int8_t*>(a.giq);
   p.gis = a.gis;
@@ -213,6 +230,8 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   p.ld_yqt = a.ld_yqt;
   p.y = static_cast<uint8_t*>(a.y);
   p.ld_y = a.ld_y;
+  p.gys = static_cast<const float*>(a.gys);
+  p.ld_gys = a.ld_gys;
   p.ld_yst = a.ld_yst;
   p.num_tiles = p.Mg * p.Kg;
   p.yqt_vec16 = (a.ld_yqt % 16 == 0) ? 1 : 0;
@@ -232,7 +251,7 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format, a.y != nullptr), mgate, mup, mdy, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(group_size, format, a.y != nullptr, qdy), mgate, mup, mdy, p);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -369,6 +388,41 @@ int sdq_fuse_strided(const void* gate, int64_t ld_gate, const void* up, int64_t 
   if (st != SDQ_OK || M == 0) return st;
   const Arrays a = {gate, ld_gate, up, ld_up, grad_y, ld_grad_y, grad_input_q, ld_grad_input_q,
                     grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y};
+  return launch(a, M, K, group_size, format, static_cast<cudaStream_t>(stream));
+}
+
+int sdq_validate_int8_grad_y(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                             const void* grad_y_q, int64_t ld_grad_y_q, const float* grad_y_s,
+                             int64_t ld_grad_y_s, const void* grad_input_q, int64_t ld_grad_input_q,
+                             const void* grad_input_s, int64_t ld_grad_input_s, const void* y_q_t,
+                             int64_t ld_y_q_t, const void* y_s_t, int64_t ld_y_s_t, const void* y,
+                             int64_t ld_y, int64_t M, int64_t K, int32_t group_size,
+                             uint32_t format) {
+  const int st = sdq_validate_strided(gate, ld_gate, up, ld_up, grad_y_q, ld_grad_y_q, grad_input_q,
+                                      ld_grad_input_q, grad_input_s, ld_grad_input_s, y_q_t,
+                                      ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y, M, K, group_size, format);
+  if (st != SDQ_OK || M == 0) return st;
+  if (!grad_y_s) return SDQ_ERR_NULL;
+  if (ld_grad_y_s < K / SDQ_GROUP_SIZE || ld_grad_y_s > SDQ_MAX_LD) return SDQ_ERR_STRIDE;
+  // code rows start on 16 bytes (tensor-map stride); scales are fp32
+  if ((ld_grad_y_q & 15) || (reinterpret_cast<uintptr_t>(grad_y_s) & 3u)) return SDQ_ERR_ALIGN;
+  return SDQ_OK;
+}
+
+int sdq_fuse_int8_grad_y(const void* gate, int64_t ld_gate, const void* up, int64_t ld_up,
+                         const void* grad_y_q, int64_t ld_grad_y_q, const float* grad_y_s,
+                         int64_t ld_grad_y_s, void* grad_input_q, int64_t ld_grad_input_q,
+                         void* grad_input_s, int64_t ld_grad_input_s, void* y_q_t, int64_t ld_y_q_t,
+                         void* y_s_t, int64_t ld_y_s_t, void* y, int64_t ld_y, int64_t M, int64_t K,
+                         int32_t group_size, uint32_t format, void* stream) {
+  const int st = sdq_validate_int8_grad_y(gate, ld_gate, up, ld_up, grad_y_q, ld_grad_y_q, grad_y_s,
+                                          ld_grad_y_s, grad_input_q, ld_grad_input_q, grad_input_s,
+                                          ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y,
+                                          M, K, group_size, format);
+  if (st != SDQ_OK || M == 0) return st;
+  const Arrays a = {gate, ld_gate, up, ld_up, grad_y_q, ld_grad_y_q, grad_input_q, ld_grad_input_q,
+                    grad_input_s, ld_grad_input_s, y_q_t, ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y,
+                    grad_y_s, ld_grad_y_s};
   return launch(a, M, K, group_size, format, static_cast<cudaStream_t>(stream));
 }
 

@@ -58,6 +58,7 @@ constexpr int kStageRows = 64;                      // token rows per pipeline s
 constexpr int kStagesPerTile = kG / kStageRows;     // 2
 constexpr int kBoxBytes = kStageRows * kG * 2;      // one bf16 box: 16 KB
 constexpr int kStageBytes = 3 * kBoxBytes;          // gate + up + grad_y
+constexpr int kQBoxBytes = kStageRows * kG;         // one INT8 grad_y box: 8 KB
 constexpr int kYBytes = kG * kG * 2;                // bf16 y tile: 32 KB
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
@@ -88,6 +89,8 @@ struct Params {
   int32_t gis_cols;  // 2K / group size: columns of grad_input_s (d_up groups from gis_cols/2)
   uint8_t* y;        // optional bf16 y [M, K] (kernels built with kY)
   int64_t ld_y;
+  const float* gys;  // INT8 grad_y's scales [M, K/128] (kernels built with kQdy)
+  int64_t ld_gys;
   int64_t ld_yqt;    // elements from one row of each output to the next
   int64_t ld_yst;
   int32_t ld_giq;    // (at most 2^24: a tile's row offsets stay 32-bit products)
@@ -140,7 +143,7 @@ __device__ __forceinline__ void tile_ij(int t, int Mg, int Kg, int& i, int& j) {
 // Load n of this CTA: stage n % 2 of its (n / 2)-th tile, into slot n % STAGES.
 // The three input tensor maps (gate, up, grad_y: [M, K] bf16 each, with their
 // own row strides; gate and up may be the two halves of one x = [gate | up]).
-template <int STAGES>
+template <int STAGES, bool kQdy>
 __device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* mgate,
                                            const CUtensorMap* mup, const CUtensorMap* mdy,
                                            const Params& p, uint32_t n, uint64_t pol) {
@@ -150,7 +153,7 @@ __device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* m
   const int r = i * kG + static_cast<int>(n % kStagesPerTile) * kStageRows;
   const uint32_t slot = n % STAGES;
   const uint32_t fb = smem_u32(&s.full[slot]);
-  mbar_arrive_expect_tx(fb, kStageBytes);
+  mbar_arrive_expect_tx(fb, kQdy ? 2 * kBoxBytes + kQBoxBytes : kStageBytes);
   const uint32_t dst = smem_u32(s.ring[slot]);
   tma_load_2d(dst, mgate, fb, j * kG, r, pol);
   tma_load_2d(dst + kBoxBytes, mup, fb, j * kG, r, pol);
@@ -163,10 +166,10 @@ __device__ __forceinline__ float2 unpack2(uint32_t v) { return make_float2(bf16_
 // Two elements: y = silu(g)*u, d_gate = dy*u*silu'(g), d_up = dy*silu(g) in
 // fp32 (packed pairs), with silu'(g) = sigma(g)*(1 + g*(1 - sigma(g)))
 // = silu*(1 - sigma) + sigma.  Results as bf16 pairs.
-__device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t dw, uint32_t& y,
-                                            uint32_t& dg, uint32_t& du) {
+__device__ __forceinline__ void swiglu_bwd2f(uint32_t gw, uint32_t uw, float2 dy, uint32_t& y,
+                                             uint32_t& dg, uint32_t& du) {
   constexpr float kNegLog2e = -1.4426950408889634f;  // e^-g = 2^(-g log2 e)
-  const float2 g = unpack2(gw), u = unpack2(uw), dy = unpack2(dw);
+  const float2 g = unpack2(gw), u = unpack2(uw);
   const float2 one = make_float2(1.0f, 1.0f);
   const float2 xl = __fmul2_rn(g, make_float2(kNegLog2e, kNegLog2e));
   const float2 d = __fadd2_rn(make_float2(ex2_approx(xl.x), ex2_approx(xl.y)), one);
@@ -180,6 +183,32 @@ __device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t d
   y = pack_bf16x2(yy.x, yy.y);
   dg = pack_bf16x2(gg.x, gg.y);
   du = pack_bf16x2(uu.x, uu.y);
+}
+
+__device__ __forceinline__ void swiglu_bwd2(uint32_t gw, uint32_t uw, uint32_t dw, uint32_t& y,
+                                            uint32_t& dg, uint32_t& du) {
+  swiglu_bwd2f(gw, uw, unpack2(dw), y, dg, du);
+}
+
+// Eight INT8 codes (channel order) times their group's scale: four fp32
+// pairs, each product rounded once.  A code c becomes a float without the
+// quarter-rate integer conversion: c + 128 (the byte XOR 0x80) placed in the
+// low mantissa byte of 2^23 is the float 2^23 + 128 + c, and subtracting
+// 2^23 + 128 leaves c exactly.
+__device__ __forceinline__ void dequant8(uint2 q, float sc, float2* out) {
+  constexpr float kBias = 8388736.0f;   // 2^23 + 128
+  const float2 s2 = make_float2(sc, sc);
+  const float2 nb = make_float2(-kBias, -kBias);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t w = (h ? q.y : q.x) ^ 0x80808080u;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {   // bytes 2p, 2p+1 into the low byte of 0x4B000000 (2^23)
+      const float lo = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (2 * p)));
+      const float hi = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (2 * p + 1)));
+      out[2 * h + p] = __fmul2_rn(__fadd2_rn(make_float2(lo, hi), nb), s2);
+    }
+  }
 }
 
 // Scale and inverse scale of a group from its amax, given as non-negative
@@ -417,7 +446,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   }
 }
 
-template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK, bool kY>
+template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK, bool kY, bool kQdy>
 __global__ void __launch_bounds__(kThreads, 1)
     fuse_kernel(const __grid_constant__ CUtensorMap map_gate, const __grid_constant__ CUtensorMap map_up,
                 const __grid_constant__ CUtensorMap map_gy,
@@ -462,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t first = total < STAGES ? total : STAGES;
     s.issued = static_cast<int>(first);
     for (uint32_t n = 0; n < first; ++n)
-      if (n != 0 || !p.withhold_first_load) issue_load(s, &map_gate, &map_up, &map_gy, p, n, pol);
+      if (n != 0 || !p.withhold_first_load)
+        issue_load<STAGES, kQdy>(s, &map_gate, &map_up, &map_gy, p, n, pol);
   }
   grid_dependency_wait();   // every thread: global memory only after the previous grid is done
   grid_launch_dependents();
@@ -503,25 +533,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int sub = 0; sub < kStagesPerTile; ++sub) {
       const uint32_t n = static_cast<uint32_t>(k) * kStagesPerTile + sub;
       const uint32_t slot = n % STAGES;
+      float dsc = 0.0f;   // INT8 grad_y: the scale of this lane's row in tile column j
+      if constexpr (kQdy) {
+        const int r = sub * kStageRows + srow;
+        if (r < valid) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + j);
+      }
       ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
       if (!ok) break;
 
       // ---- stage -> registers, then release the slot (the last warp refills it)
       uint32_t gw[8], uw[8], dw[8];
+      float2 dq[8];   // INT8 grad_y, dequantized
       {
         const uint8_t* src = s.ring[slot] + srow * (kG * 2);
         const uint4 g0 = *reinterpret_cast<const uint4*>(src + ca * 16);
         const uint4 g1 = *reinterpret_cast<const uint4*>(src + cb * 16);
         const uint4 u0 = *reinterpret_cast<const uint4*>(src + kBoxBytes + ca * 16);
         const uint4 u1 = *reinterpret_cast<const uint4*>(src + kBoxBytes + cb * 16);
-        const uint4 d0 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + ca * 16);
-        const uint4 d1 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + cb * 16);
         gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
         gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
         uw[0] = u0.x; uw[1] = u0.y; uw[2] = u0.z; uw[3] = u0.w;
         uw[4] = u1.x; uw[5] = u1.y; uw[6] = u1.z; uw[7] = u1.w;
-        dw[0] = d0.x; dw[1] = d0.y; dw[2] = d0.z; dw[3] = d0.w;
-        dw[4] = d1.x; dw[5] = d1.y; dw[6] = d1.z; dw[7] = d1.w;
+        if constexpr (kQdy) {   // codes of row srow: 128 bytes, 8 per chunk
+          const uint8_t* qsrc = s.ring[slot] + 2 * kBoxBytes + srow * kG;
+          dequant8(*reinterpret_cast<const uint2*>(qsrc + ca * 8), dsc, dq);
+          dequant8(*reinterpret_cast<const uint2*>(qsrc + cb * 8), dsc, dq + 4);
+        } else {
+          const uint4 d0 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + ca * 16);
+          const uint4 d1 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + cb * 16);
+          dw[0] = d0.x; dw[1] = d0.y; dw[2] = d0.z; dw[3] = d0.w;
+          dw[4] = d1.x; dw[5] = d1.y; dw[6] = d1.z; dw[7] = d1.w;
+        }
       }
       __syncwarp();
       if (lane == 0) {
@@ -532,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t nn = n + STAGES;
           if (nn < total) {
             atomicMax(&s.issued, static_cast<int>(nn + 1));
-            issue_load(s, &map_gate, &map_up, &map_gy, p, nn, pol);
+            issue_load<STAGES, kQdy>(s, &map_gate, &map_up, &map_gy, p, nn, pol);
           }
         }
       }
@@ -540,7 +582,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- math, bf16 rounding
       uint32_t yv[8], dgp[8], dup[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) swiglu_bwd2(gw[c], uw[c], dw[c], yv[c], dgp[c], dup[c]);
+      for (int c = 0; c < 8; ++c) {
+        if constexpr (kQdy) swiglu_bwd2f(gw[c], uw[c], dq[c], yv[c], dgp[c], dup[c]);
+        else swiglu_bwd2(gw[c], uw[c], dw[c], yv[c], dgp[c], dup[c]);
+      }
 
       // ---- y to the shared tile (chunks swizzled by token); the buffer was
       // last read by the column pass of tile k - kYBuf

@@ -230,3 +230,35 @@ def test_fwd_rejects_bad_arguments_without_launching():
     assert sdq.sdq_validate_swiglu_q8_1(A + 2, 64, A, 64, None, A, 64, A, 4, 64) == sdq.Status.ERR_ALIGN
     assert sdq.sdq_validate_swiglu_q8_1(A, 64, A, 64, None, A, 64, A + 2, 4, 64) == sdq.Status.ERR_ALIGN
     assert sdq.sdq_validate_swiglu_q8_1(0, 64, 0, 64, None, 0, 64, 0, 0, 64) == sdq.Status.OK
+
+
+def _int8_gy_args(**kw):
+    M, K = 256, 256
+    a = dict(gate=A, ld_gate=2 * K, up=A + 2 * K, ld_up=2 * K, grad_y_q=A, ld_grad_y_q=K,
+             grad_y_s=A, ld_grad_y_s=2, grad_input_q=A, ld_grad_input_q=2 * K, grad_input_s=A,
+             ld_grad_input_s=4, y_q_t=A, ld_y_q_t=M, y_s_t=A, ld_y_s_t=2, y=None, ld_y=0, M=M, K=K,
+             group_size=128, format=0)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0),
+    (dict(ld_grad_y_q=272, ld_grad_y_s=5), 0),          # padded rows
+    (dict(ld_grad_y_q=264), 4),                          # code rows must start on 16 bytes
+    (dict(ld_grad_y_q=255), 10),
+    (dict(grad_y_q=A + 8), 4),
+    (dict(grad_y_s=None), 1),
+    (dict(grad_y_q=None), 1),
+    (dict(ld_grad_y_s=1), 10),                           # fewer than K/128 scales a row
+    (dict(ld_grad_y_s=(1 << 36) + 1), 10),
+    (dict(grad_y_s=A + 2), 4),                           # fp32 scales on 4 bytes
+    (dict(grad_y_s=A + 4), 0),
+    (dict(y=A, ld_y=256, format=7, ld_y_s_t=256), 0),    # with y, another format
+    (dict(M=0, gate=None, up=None, grad_y_q=None, grad_y_s=None), 0),
+    (dict(group_size=96), 2),
+])
+def test_validate_int8_grad_y_statuses(kw, status):
+    import swiglu_backward_int8_b200 as sdq
+    a = _int8_gy_args(**kw)
+    assert sdq.sdq_validate_int8_grad_y(*a.values()) == status
