@@ -120,3 +120,45 @@ def test_wrapper_takes_int8_grad_y():
         sdq.silu_dot_fwd_bwd_quant_fuse(xd, qd.to(torch.bfloat16), *outs, grad_y_s=sd)
     with pytest.raises(ValueError):
         sdq.silu_dot_fwd_bwd_quant_fuse(xd, qd, *outs, grad_y_s=sd[:, :1])
+
+
+@pytest.mark.slow
+def test_int8_grad_y_full_size_sampled_tiles():
+    """M=16384, K=7168 in one launch with grad_y as INT8 codes + scales and the
+    bf16 y written too: 24 sampled 128x128 tiles against the oracle on each
+    tile (every group lies inside one tile, and so does each row's scale of
+    the tile's 128 grad_y channels); y on the same tiles."""
+    import swiglu_backward_int8_b200 as sdq
+    w = W.WORKLOADS[4]
+    M, K = w.M, w.K
+    x, _ = W.make_inputs(w)
+    q, s = W.quantized_grad_y(w)
+    outs = sdq.allocate_outputs(M, K, "cuda")
+    y = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse(U.to_device_bf16(x), torch.from_numpy(q).cuda(), *outs, y=y,
+                                    grad_y_s=torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    assert sdq.sdq_device_status() == 0
+    giq, gis, yqt, yst = (t.cpu().numpy() for t in outs)
+    yh = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    rng = np.random.default_rng(11)
+    tiles = {(0, 0), (M // 128 - 1, K // 128 - 1)}
+    while len(tiles) < 24:
+        tiles.add((int(rng.integers(M // 128)), int(rng.integers(K // 128))))
+    n_diff = 0
+    for i, j in sorted(tiles):
+        r0, c0 = 128 * i, 128 * j
+        xt = np.concatenate([x[r0:r0 + 128, c0:c0 + 128], x[r0:r0 + 128, K + c0:K + c0 + 128]], axis=1)
+        qt, st_ = q[r0:r0 + 128, c0:c0 + 128], s[r0:r0 + 128, j:j + 1]
+        ref = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(xt, qt, st_, 128, 0, 0, 0)
+        got = (np.concatenate([giq[r0:r0 + 128, c0:c0 + 128], giq[r0:r0 + 128, K + c0:K + c0 + 128]],
+                              axis=1).view(np.uint8),
+               np.stack([gis[r0:r0 + 128, j], gis[r0:r0 + 128, K // 128 + j]], axis=1),
+               yqt[c0:c0 + 128, r0:r0 + 128].view(np.uint8), yst[c0:c0 + 128, i:i + 1])
+        st = U.compare_fmt(got, ref, 0, 0, 0, f"M16384 INT8 grad_y tile ({i},{j})", 128,
+                           max_frac=1.0)                 # the 0.1 % bound applies to the whole sample
+        n_diff += st["grad_input_q"]["n_diff"] + st["y_q_t"]["n_diff"]
+        ry = oracle.swiglu_bwd_bf16_dy(xt, oracle.dequant_grad_y(qt, st_))[0]
+        U.compare_bf16(yh[r0:r0 + 128, c0:c0 + 128], ry, "y", f"tile ({i},{j})")
+    total = 24 * 128 * 128 * 3
+    assert n_diff <= 1e-3 * total, f"{n_diff} of {total} sampled codes differ"
