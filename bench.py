@@ -31,6 +31,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -97,11 +98,22 @@ def pick_workload(name: str) -> W.Workload:
     return W.BY_NAME[name]
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without comments and blank-line or trailing-space
+    differences (no string literal in these sources holds a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_sha(sources=None) -> str:
+    """Digest of a kernel's sources, comments excluded: a profile recorded
+    under it stays valid across comment-only edits and lapses with any code
+    change."""
     h = hashlib.sha256()
     for f in (sources or KERNEL_SOURCES):
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

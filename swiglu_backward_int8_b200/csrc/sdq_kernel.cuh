@@ -7,6 +7,13 @@
 //   grad_input_q/_s: [d_gate | d_up] quantized per token in 128-channel groups,
 //   y_q_t/_s_t:      y transposed, quantized per channel in 128-token groups.
 //
+// Template variants (each its own instantiation, so a variant's work never
+// reaches the others): group size 128, 64 or 32 (a tile holds whole groups
+// of each); code format INT8 or FP8 E4M3, scale format fp32 or E8M0, y_s_t
+// [K, Mg] or [Mg, K]; kY, the recomputed bf16 y also stored from registers;
+// kQdy, grad_y read as INT8 codes (an 8-bit box in the stage's third slot)
+// times one fp32 scale per token and 128 channels.
+//
 // Work decomposition.  A 128-token x 128-channel tile (i, j) holds exactly one
 // quantization group on both axes, so tiles are independent.  The grid is
 // persistent (at most one CTA per SM); CTA b walks tiles b, b + grid, ... in a
@@ -26,9 +33,9 @@
 //   * row pass: a lane owns 16 channels of one token row per stage (8 lanes per
 //     row, 4 rows per warp): fp32 math in packed f32x2 instructions, bf16
 //     rounding, the row amax of d_gate and d_up by a 3-step shuffle reduction
-//     on packed bf16 pairs, the warp's 8 row scales computed by lanes 0-7 at
-//     once and shuffled back, quantization by multiplication with the inverse
-//     scale, coalesced stores; the bf16 y values go to a shared [token][channel]
+//     on packed bf16 pairs, each lane computing its row's two scales itself
+//     (no shuffles), quantization by multiplication with the inverse scale,
+//     coalesced stores; the bf16 y values go to a shared [token][channel]
 //     tile (double-buffered across tiles).
 //   * column pass, one tile late (after the row pass of the next tile, so no
 //     warp waits for the others at a tile boundary; two mbarriers per y buffer
