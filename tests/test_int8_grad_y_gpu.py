@@ -162,3 +162,18 @@ def test_int8_grad_y_full_size_sampled_tiles():
         U.compare_bf16(yh[r0:r0 + 128, c0:c0 + 128], ry, "y", f"tile ({i},{j})")
     total = 24 * 128 * 128 * 3
     assert n_diff <= 1e-3 * total, f"{n_diff} of {total} sampled codes differ"
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (31, 128), (127, 256), (257, 128), (640, 640)])
+def test_int8_grad_y_odd_shapes_with_y(M, K):
+    """Tail token groups of 1..127 tokens, M % 16 != 0 (byte-wise y_q_t
+    stores), one channel tile: outputs against the oracle, y against the
+    oracle's first stage."""
+    w = W.small_workload(M, K, seed=3 * M + K, zero_group_every=5)
+    x, _ = W.make_inputs(w)
+    q, s = W.quantized_grad_y(w)
+    got = _run_int8_grad_y(x, q, s, 128, (0, 0, 0), pad=1, with_y=True)
+    ref = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, 128, 0, 0, 0)
+    U.compare_fmt(got[:4], ref, 0, 0, 0, f"int8 grad_y M={M} K={K}", 128)
+    U.compare_bf16(got[4], oracle.swiglu_bwd_bf16_dy(x, oracle.dequant_grad_y(q, s))[0], "y",
+                   f"M={M} K={K}")
