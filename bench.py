@@ -21,6 +21,9 @@ e2e   = the same metric through the host-buffer entry point (sdq_fuse_host):
         pinned host memory, every step inside the timed region.
 cpu_baseline / --impl reference = the CPU oracle (single thread) timed on
         bounded samples of the same workload.
+with_y / int8_grad_y = side measurements on the same workload: the call that
+        also writes the bf16 y, and the call with grad_y as INT8 codes + fp32
+        scales (skipped with --no-variants).
 
 Multi-GPU (torchrun): each rank runs an independent replica of the workload
 (the op has no exchange step; weak scaling); NCCL carries only the barrier
@@ -79,9 +82,14 @@ def parse_args():
                          "SwiGLU + q8_1 rows on the workload's gate and up (rows = M, inter = K)")
     ap.add_argument("--limit", type=float, default=0.0, help="swiglu_q8_1: the clamp (0: none)")
     ap.add_argument("--int8-grad-y", action="store_true",
-                    help="also time the call with grad_y given as INT8 codes + fp32 scales")
+                    help="also time the call with grad_y given as INT8 codes + fp32 scales "
+                         "(on by default; see --no-variants)")
     ap.add_argument("--with-y", action="store_true",
-                    help="also time the call with the optional bf16 y output")
+                    help="also time the call with the optional bf16 y output (on by default; "
+                         "see --no-variants)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the side measurements of the y output and the INT8 grad_y input "
+                         "unless asked for by --with-y / --int8-grad-y")
     ap.add_argument("--all-formats", action="store_true",
                     help="also time every output format on the workload and add a per_format list")
     a = ap.parse_args()
@@ -469,7 +477,7 @@ def run_sdq(args):
                                     "algorithmic_bytes_per_launch": fb})
 
     with_y = None
-    if args.with_y:   # the same call also writing the optional bf16 y
+    if args.with_y or not args.no_variants:   # the same call also writing the optional bf16 y
         yms, _, _ = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, with_y=True)
         yms = parallel.max_over_ranks(yms, device)
         us = yms / args.steps * 1e3
@@ -479,7 +487,7 @@ def run_sdq(args):
                   "algorithmic_bytes_per_launch": yb, "format": format_name(PAGE_FORMAT)}
 
     int8_gy = None
-    if args.int8_grad_y:   # grad_y handed over as INT8 codes + fp32 scales
+    if args.int8_grad_y or not args.no_variants:   # grad_y handed over as INT8 codes + fp32 scales
         qgy = W.quantized_grad_y(wr)
         qms, _, _ = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device,
                                    int8_grad_y=qgy)
