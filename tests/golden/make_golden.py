@@ -55,10 +55,29 @@ def record(w: W.Workload) -> dict:
     }
 
 
+# grad_y handed over as INT8 codes + fp32 scales (workloads.quantized_grad_y)
+QGRAD_CASES = [W.small_workload(200, 384, seed=5, zero_group_every=7),
+               W.small_workload(129, 256, seed=11, zero_group_every=3)]
+
+
+def record_qgrad(w: W.Workload) -> dict:
+    x, _ = W.make_inputs(w)
+    q, s = W.quantized_grad_y(w)
+    outs = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, w.group_size)
+    y = oracle.swiglu_bwd_bf16_dy(x, oracle.dequant_grad_y(q, s))[0]
+    names = ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")
+    return {
+        "workload": w.describe(),
+        "inputs_sha256": {"x": digest(x), "grad_y_q": digest(q), "grad_y_s": digest(s)},
+        "outputs_sha256": dict({n: digest(a) for n, a in zip(names, outs)}, y=digest(y)),
+    }
+
+
 def main() -> None:
     out = {"source": "CPU oracle (oracle/sdq_oracle.cpp) on workloads.make_inputs; "
                      "regression record only, not a pin",
-           "cases": [record(w) for w in CASES]}
+           "cases": [record(w) for w in CASES],
+           "qgrad_cases": [record_qgrad(w) for w in QGRAD_CASES]}
     with open(os.path.join(HERE, "oracle_records.json"), "w") as f:
         json.dump(out, f, indent=1)
         f.write("\n")

@@ -10,7 +10,7 @@ import numpy as np
 
 import oracle
 import workloads as W
-from tests.golden.make_golden import CASES, digest
+from tests.golden.make_golden import CASES, QGRAD_CASES, digest, record_qgrad
 
 HERE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -34,3 +34,10 @@ def test_oracle_matches_regression_records():
             assert float(gis[m, j]) == v
         for k, i, v in r["samples"]["y_s_t"]:
             assert float(yst[k, i]) == v
+
+
+def test_quantized_grad_y_oracle_matches_regression_records():
+    rec = json.load(open(os.path.join(HERE, "oracle_records.json")))
+    assert len(rec["qgrad_cases"]) == len(QGRAD_CASES)
+    for w, r in zip(QGRAD_CASES, rec["qgrad_cases"]):
+        assert record_qgrad(w) == r, w.name
