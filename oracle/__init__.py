@@ -204,8 +204,10 @@ def quant_group_fmt(v_bf16: np.ndarray, codes: int = 0, scales: int = 0):
 
 
 def output_shapes_fmt(M: int, K: int, group_size: int = 128, ys_layout: int = 0):
+    """Output shapes; with G not dividing K each half of a row ends in a
+    shorter group, so grad_input_s has 2 * ceil(K/G) columns."""
     G = int(group_size)
-    Kg, Mg = K // G, (M + G - 1) // G
+    Kg, Mg = (K + G - 1) // G, (M + G - 1) // G
     return (M, 2 * K), (M, 2 * Kg), (K, M), ((Mg, K) if ys_layout else (K, Mg))
 
 
@@ -213,17 +215,18 @@ def silu_dot_fwd_bwd_quant_fuse_fmt(x: np.ndarray, grad_y: np.ndarray, group_siz
                                     codes: int = 0, scales: int = 0, ys_layout: int = 0):
     """The whole op in a chosen output format, on uint16 (bf16 bit) arrays.
 
-    Returns ``(grad_input_q [M,2K] uint8 code bytes, grad_input_s [M,2K/G],
-    y_q_t [K,M] uint8, y_s_t [K,Mg] or [Mg,K])``; scale arrays are float32
-    (fp32 scales) or uint8 (E8M0 bytes).
+    Returns ``(grad_input_q [M,2K] uint8 code bytes, grad_input_s
+    [M,2*ceil(K/G)], y_q_t [K,M] uint8, y_s_t [K,Mg] or [Mg,K])``; scale
+    arrays are float32 (fp32 scales) or uint8 (E8M0 bytes).  When G does not
+    divide K, each half of [d_gate | d_up] ends in a shorter group.
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     gy = np.ascontiguousarray(grad_y, dtype=np.uint16)
     M, K = gy.shape
     assert x.shape == (M, 2 * K), (x.shape, gy.shape)
     G = int(group_size)
-    if G < 1 or K % G:
-        raise ValueError(f"K={K} is not a multiple of group_size={G}")
+    if G < 1:
+        raise ValueError(f"group_size={G}")
     sq, ss, yq, ys = output_shapes_fmt(M, K, G, ys_layout)
     sdt = np.uint8 if scales else np.float32
     giq = np.zeros(sq, np.uint8)
@@ -247,7 +250,7 @@ def dequant_grad_y(grad_y_q: np.ndarray, grad_y_s: np.ndarray) -> np.ndarray:
     q = np.ascontiguousarray(grad_y_q, dtype=np.int8)
     sc = np.ascontiguousarray(grad_y_s, dtype=np.float32)
     M, K = q.shape
-    assert K % 128 == 0 and sc.shape == (M, K // 128), (q.shape, sc.shape)
+    assert sc.shape == (M, (K + 127) // 128), (q.shape, sc.shape)
     dy = np.empty((M, K), np.float64)
     lib().oracle_dequant_grad_y(_ptr(q), _ptr(sc), M, K, _ptr(dy))
     return dy
@@ -275,7 +278,7 @@ def silu_dot_fwd_bwd_quant_fuse_qgrad(x: np.ndarray, grad_y_q: np.ndarray, grad_
     q = np.ascontiguousarray(grad_y_q, dtype=np.int8)
     sc = np.ascontiguousarray(grad_y_s, dtype=np.float32)
     M, K = q.shape
-    assert x.shape == (M, 2 * K) and sc.shape == (M, K // 128), (x.shape, q.shape, sc.shape)
+    assert x.shape == (M, 2 * K) and sc.shape == (M, (K + 127) // 128), (x.shape, q.shape, sc.shape)
     G = int(group_size)
     sq, ss, yq, ys = output_shapes_fmt(M, K, G, ys_layout)
     sdt = np.uint8 if scales else np.float32

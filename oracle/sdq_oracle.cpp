@@ -336,7 +336,7 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
                                            int64_t group_size, int codes, int scales,
                                            int ys_layout) {
   const int64_t G = group_size;
-  if (G < 1 || M < 0 || K < 0 || K % G != 0) return -1;
+  if (G < 1 || M < 0 || K < 0) return -1;
   if (codes < 0 || codes > 1 || scales < 0 || scales > 1 || ys_layout < 0 || ys_layout > 1) return -1;
   if (M == 0 || K == 0) return 0;
   std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
@@ -350,18 +350,19 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
 //
 // Reading: the upstream step hands grad_y over in the row-group format this
 // op itself writes for grad_input: INT8 codes q [M, K] and fp32 scales
-// s [M, K/128], one per token and 128 consecutive channels; the value it
-// stands for is q * s (exact in fp64: 8 x 24 significant bits).
+// s [M, ceil(K/128)], one per token and 128 consecutive channels (the last
+// group of a row holds what is left); the value it stands for is q * s
+// (exact in fp64: 8 x 24 significant bits).
 
 // dy[m, k] = q[m, k] * s[m, k / 128].
 void oracle_dequant_grad_y(const int8_t* q, const float* s, int64_t M, int64_t K, double* dy) {
-  const int64_t Kg = K / 128;
+  const int64_t Kg = (K + 127) / 128;
   for (int64_t m = 0; m < M; ++m)
     for (int64_t k = 0; k < K; ++k)
       dy[m * K + k] = static_cast<double>(q[m * K + k]) * static_cast<double>(s[m * Kg + k / 128]);
 }
 
-// The whole op with a quantized grad_y (K a multiple of 128), outputs as in
+// The whole op with a quantized grad_y, outputs as in
 // oracle_silu_dot_fwd_bwd_quant_fuse_fmt.
 int oracle_silu_dot_fwd_bwd_quant_fuse_qgrad(const uint16_t* x, const int8_t* grad_y_q,
                                              const float* grad_y_s, uint8_t* grad_input_q,
@@ -369,7 +370,7 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_qgrad(const uint16_t* x, const int8_t* gr
                                              int64_t M, int64_t K, int64_t group_size, int codes,
                                              int scales, int ys_layout) {
   const int64_t G = group_size;
-  if (G < 1 || M < 0 || K < 0 || K % G != 0 || K % 128 != 0) return -1;
+  if (G < 1 || M < 0 || K < 0) return -1;
   if (codes < 0 || codes > 1 || scales < 0 || scales > 1 || ys_layout < 0 || ys_layout > 1) return -1;
   if (M == 0 || K == 0) return 0;
   std::vector<double> dy(M * K);
@@ -381,12 +382,16 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_qgrad(const uint16_t* x, const int8_t* gr
   return 0;
 }
 
-// The two quantizations of the first stage's bf16 y, d_gate, d_up.
+// The two quantizations of the first stage's bf16 y, d_gate, d_up.  Row
+// groups are taken within each half of [d_gate | d_up]: ceil(K/G) groups of
+// G channels per half, the last one holding the K - (ceil(K/G) - 1) * G
+// channels left when G does not divide K; grad_input_s is [M, 2 ceil(K/G)],
+// d_gate's groups first.
 static void quantize_outputs_fmt(const uint16_t* y, const uint16_t* dg, const uint16_t* du,
                                  uint8_t* grad_input_q, void* grad_input_s, uint8_t* y_q_t,
                                  void* y_s_t, int64_t M, int64_t K, int64_t G, int codes,
                                  int scales, int ys_layout) {
-  const int64_t Kg = K / G;
+  const int64_t Kg = (K + G - 1) / G;
   const int64_t Mg = (M + G - 1) / G;
   const int64_t sb = scales ? 1 : 4;   // bytes per scale
   uint8_t* gis = static_cast<uint8_t*>(grad_input_s);
@@ -394,7 +399,9 @@ static void quantize_outputs_fmt(const uint16_t* y, const uint16_t* dg, const ui
   for (int64_t m = 0; m < M; ++m) {
     for (int64_t j = 0; j < 2 * Kg; ++j) {
       const uint16_t* src = (j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G];
-      oracle_quant_group_fmt(src, G, 1, &grad_input_q[m * 2 * K + j * G], 1,
+      const int64_t c0 = (j < Kg) ? j * G : (j - Kg) * G;   // first channel within its half
+      const int64_t n = (K - c0 < G) ? K - c0 : G;
+      oracle_quant_group_fmt(src, n, 1, &grad_input_q[m * 2 * K + (j < Kg ? 0 : K) + c0], 1,
                              gis + (m * 2 * Kg + j) * sb, codes, scales);
     }
   }

@@ -264,3 +264,33 @@ def test_whole_op_e4m3_gate32_closed_form():
     for t in range(M):
         if int(a[t]) in want:
             assert np.all(yqt[:, t] == want[int(a[t])]), t
+
+
+# ----------------------------------------------------------------------------
+# G not dividing K: each half of [d_gate | d_up] ends in a shorter group
+# ----------------------------------------------------------------------------
+
+def _pad_channels(a, K, Kp):
+    """[M, K] (or the two halves of [M, 2K]) widened to Kp channels with zeros."""
+    if a.shape[1] == K:
+        return np.concatenate([a, np.zeros((a.shape[0], Kp - K), a.dtype)], axis=1)
+    return np.concatenate([_pad_channels(a[:, :K], K, Kp), _pad_channels(a[:, K:], K, Kp)], axis=1)
+
+
+@pytest.mark.parametrize("K,G", [(200, 128), (144, 128), (208, 64), (80, 32), (16, 128), (1040, 128)])
+@pytest.mark.parametrize("fmt", [(0, 0, 0), (1, 1, 1), (0, 1, 1)])
+def test_short_last_group_equals_the_zero_padded_op(K, G, fmt):
+    """Zero channels change no amax and quantize to zero, so the op on K
+    channels equals the op on K padded with zeros to a multiple of G (where
+    every group is whole), restricted to the K real channels of each half."""
+    M = 131
+    Kp = (K + G - 1) // G * G
+    x, gy = W.make_inputs(W.small_workload(M, K, seed=K + G, zero_group_every=0))
+    got = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, G, *fmt)
+    pad = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(_pad_channels(x, K, Kp), _pad_channels(gy, K, Kp), G, *fmt)
+    assert np.array_equal(got[0], np.concatenate([pad[0][:, :K], pad[0][:, Kp:Kp + K]], axis=1))
+    assert np.array_equal(got[1], pad[1])               # ceil(K/G) groups per half either way
+    assert np.array_equal(got[2], pad[2][:K])
+    ys = pad[3][:, :K] if fmt[2] else pad[3][:K]
+    assert np.array_equal(got[3], ys)
+    assert got[1].shape == (M, 2 * ((K + G - 1) // G))

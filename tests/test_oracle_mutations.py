@@ -69,6 +69,11 @@ MUTATIONS = [
      "test_swiglu_rows_blocks_are_the_rows_32_value_blocks", "fwd"),
     ("if (limit > 0.0) {   // false for NaN: no clamp", "if (limit != 0.0) {",
      "test_swiglu_rows_closed_form_without_clamp", "fwd"),
+    # groups of G channels when G does not divide K (pins in test_oracle_formats.py)
+    ("const int64_t n = (K - c0 < G) ? K - c0 : G;", "const int64_t n = G < K ? G : K;",
+     "test_short_last_group_equals_the_zero_padded_op", "formats"),
+    ("&grad_input_q[m * 2 * K + (j < Kg ? 0 : K) + c0]", "&grad_input_q[m * 2 * K + j * G]",
+     "test_short_last_group_equals_the_zero_padded_op", "formats"),
     # a quantized grad_y (pins in test_oracle_qgrad.py)
     ("static_cast<double>(s[m * Kg + k / 128])", "static_cast<double>(s[m * Kg + k % Kg])",
      "test_whole_op_pow2_scales_equals_bf16_op", "qgrad"),

@@ -32,13 +32,13 @@ def _bf16_of_exact_f32(v: np.ndarray) -> np.ndarray:
 
 @pytest.mark.parametrize("G", [128, 64, 32])
 @pytest.mark.parametrize("fmt", [(0, 0, 0), (1, 1, 1), (0, 1, 1), (1, 0, 0)])
-@pytest.mark.parametrize("M,K", [(300, 384), (129, 256)])
+@pytest.mark.parametrize("M,K", [(300, 384), (129, 256), (129, 208)])
 def test_whole_op_pow2_scales_equals_bf16_op(M, K, G, fmt):
     w = W.small_workload(M, K, seed=M + K + G, zero_group_every=7)
     x, _ = W.make_inputs(w)
     q, s = W.quantized_grad_y(w, pow2_scales=True)
     assert len(np.unique(s)) > 3 and (s[:, :, None] != s[:1, :1, None]).any()
-    gy = _bf16_of_exact_f32(q.astype(np.float32) * np.repeat(s, 128, axis=1))
+    gy = _bf16_of_exact_f32(q.astype(np.float32) * np.repeat(s, 128, axis=1)[:, :K])
     got = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, G, *fmt)
     ref = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, G, *fmt)
     for a, b, name in zip(got, ref, ("grad_input_q", "grad_input_s", "y_q_t", "y_s_t")):
@@ -75,8 +75,11 @@ def test_dequant_is_exact_in_fp64():
     assert np.array_equal(back, q.astype(np.float64))
 
 
-def test_qgrad_rejects_uncovered_shapes():
-    x = np.zeros((4, 2 * 64), np.uint16)
-    with pytest.raises(ValueError):         # K = 64: no 128-channel scale groups
-        oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, np.zeros((4, 64), np.int8),
-                                                 np.zeros((4, 0), np.float32))
+def test_qgrad_short_last_scale_group():
+    """K = 200: a row's second scale covers its last 72 channels only."""
+    w = W.small_workload(16, 200, seed=13)
+    q, s = W.quantized_grad_y(w)
+    assert s.shape == (16, 2)
+    dy = oracle.dequant_grad_y(q, s)
+    assert np.array_equal(dy[:, 128:], q[:, 128:].astype(np.float64) * s[:, 1:2].astype(np.float64))
+    assert np.array_equal(dy[:, :128], q[:, :128].astype(np.float64) * s[:, :1].astype(np.float64))

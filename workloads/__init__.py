@@ -256,14 +256,14 @@ STREAM_GRAD_Y_SCALES = 9
 
 def quantized_grad_y(w: Workload, pow2_scales: bool = False):
     """A grad_y already in the row-group INT8 format: (codes int8 [M, K],
-    scales float32 [M, K/128]).  Codes are a normal of spread 42 rounded and
+    scales float32 [M, ceil(K/128)]).  Codes are a normal of spread 42 rounded and
     clipped to [-127, 127] (one value per channel); scales are
     sigma_grad_y / 42 times a log-normal factor exp(N(0, 1/4)) per token and
     128-channel group, so the values have about the bf16 grad_y's spread;
     with ``pow2_scales`` each scale is the nearest power of two of that.
     Every ``zero_group_every``-th token has one all-zero code group."""
     M, K = w.M, w.K
-    Kg = K // 128
+    Kg = (K + 127) // 128   # the last scale of a row covers what is left of it
     z = normals(stream_key(w.seed, STREAM_GRAD_Y_CODES), 0, M * K)
     q = np.clip(np.rint(z * 42.0), -127, 127).astype(np.int8).reshape(M, K)
     e = normals(stream_key(w.seed, STREAM_GRAD_Y_SCALES), 0, M * Kg).reshape(M, Kg)
