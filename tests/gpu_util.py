@@ -222,7 +222,13 @@ def compare_fmt(got, ref, codes: int, scales: int, ys_layout: int, where="", gro
             assert rel.max(initial=0) <= SCALE_MAX_REL, f"{where} {name}: max rel = {rel.max()}"
     G = group_size
     M = giq.shape[0]
-    for name, a, b, sa, sb in (("grad_input_q", giq, rq, np.repeat(gis, G, axis=1), np.repeat(rs, G, axis=1)),
+    K = giq.shape[1] // 2
+    # each code's row scale: channel c of [d_gate | d_up] is in group
+    # half * ceil(K/G) + (c mod K) // G (a half may end in a shorter group)
+    Kgs = (K + G - 1) // G
+    c = np.arange(2 * K)
+    col = (c // K) * Kgs + (c % K) // G
+    for name, a, b, sa, sb in (("grad_input_q", giq, rq, gis[:, col], rs[:, col]),
                                ("y_q_t", yqt, ryq, np.repeat(yst, G, axis=1)[:, :M],
                                 np.repeat(rys, G, axis=1)[:, :M])):
         assert a.shape == b.shape, (name, a.shape, b.shape)
