@@ -40,6 +40,13 @@ def _worker(rank: int, world: int, port: int, M: int, K: int) -> None:
         mine = oracle.silu_dot_fwd_bwd_quant_fuse(x[m0:m1], gy[m0:m1])
         ok = (np.array_equal(mine[0], full[0][m0:m1]) and np.array_equal(mine[1], full[1][m0:m1])
               and np.array_equal(mine[2], full[2][:, m0:m1]) and np.array_equal(mine[3], full[3][:, i0:i1]))
+        # the same with grad_y handed over as INT8 codes + scales (their rows shard with the tokens)
+        q, sc = W.quantized_grad_y(w)
+        qfull = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, sc)
+        qmine = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x[m0:m1], q[m0:m1], sc[m0:m1])
+        ok = ok and (np.array_equal(qmine[0], qfull[0][m0:m1]) and np.array_equal(qmine[1], qfull[1][m0:m1])
+                     and np.array_equal(qmine[2], qfull[2][:, m0:m1])
+                     and np.array_equal(qmine[3], qfull[3][:, i0:i1]))
         flag = torch.tensor([1 if ok else 0], dtype=torch.int32)
         dist.all_reduce(flag, op=dist.ReduceOp.MIN)
         assert flag.item() == 1, f"rank {rank}: shard result differs from the global result"
