@@ -69,6 +69,11 @@ MUTATIONS = [
      "test_swiglu_rows_blocks_are_the_rows_32_value_blocks", "fwd"),
     ("if (limit > 0.0) {   // false for NaN: no clamp", "if (limit != 0.0) {",
      "test_swiglu_rows_closed_form_without_clamp", "fwd"),
+    # the whole op against its brute-force restatement (test_oracle_bruteforce.py)
+    ("*d_up = dy * silu;", "*d_up = dy * silu * u;", "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
+    ("x[m * 2 * K + k]);", "x[m * 2 * K + K + k]);", "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
+    ("const float s = amax / 127.0f;", "const float s = amax / 127.5f;",
+     "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
     # groups of G channels when G does not divide K (pins in test_oracle_formats.py)
     ("const int64_t n = (K - c0 < G) ? K - c0 : G;", "const int64_t n = G < K ? G : K;",
      "test_short_last_group_equals_the_zero_padded_op", "formats"),
@@ -87,7 +92,8 @@ MUTATIONS = [
 ]
 
 PIN_FILES = {"pins": "test_oracle_pins.py", "formats": "test_oracle_formats.py",
-             "fwd": "test_oracle_fwd.py", "qgrad": "test_oracle_qgrad.py"}
+             "fwd": "test_oracle_fwd.py", "qgrad": "test_oracle_qgrad.py",
+             "brute": "test_oracle_bruteforce.py"}
 
 
 def _run_mutant(tmp_dir, idx, old, new, pin, pins="pins"):
