@@ -277,7 +277,7 @@ def _pad_channels(a, K, Kp):
     return np.concatenate([_pad_channels(a[:, :K], K, Kp), _pad_channels(a[:, K:], K, Kp)], axis=1)
 
 
-@pytest.mark.parametrize("K,G", [(200, 128), (144, 128), (208, 64), (80, 32), (16, 128), (1040, 128)])
+@pytest.mark.parametrize("K,G", [(200, 128), (144, 128), (208, 64), (80, 32), (16, 128), (1040, 128), (384, 256)])
 @pytest.mark.parametrize("fmt", [(0, 0, 0), (1, 1, 1), (0, 1, 1)])
 def test_short_last_group_equals_the_zero_padded_op(K, G, fmt):
     """Zero channels change no amax and quantize to zero, so the op on K
