@@ -2,17 +2,21 @@
 """Benchmark of silu_dot_fwd_bwd_quant_fuse on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdq|reference]
-                    [--workload NAME|INDEX] [--all-workloads] [--no-cpu-baseline]
+                    [--workload NAME|INDEX] [--no-per-workload] [--no-cpu-baseline]
 
 One step = one call of the fused op over one synthetic batch of the
-workload (default: M=4096 tokens, K=1408 channels, the MoE-expert-sized FFN).
-Prints ONE JSON line on rank 0.
+workload (default: M=16384 tokens, K=7168 channels, the bandwidth-roofline
+case and the largest of the five workloads).  Prints ONE JSON line on rank 0;
+besides the headline it carries a per_workload list timing all five
+workloads (skipped with --no-per-workload).
 
 Timing: W eager warm-up calls, then EXACTLY K calls replayed from CUDA
 graphs, bracketed by a barrier and a device synchronize and timed with CUDA
 events on the launching stream; the maximum over ranks is taken.  Between
 consecutive calls the inputs and outputs rotate through enough buffer sets to
-exceed 3x the L2 cache, so no call finds its data in L2.
+exceed 3x the L2 cache, so no call finds its data in L2 (a call of the
+default workload moves 1.07 GB, so one set does).  The per_workload entries
+time each workload for at least about 50 ms of calls.
 
 value = algorithmic bytes of all ranks / time (GB/s); the algorithmic bytes
 are 6 B read + 3 B written per (token, channel) plus the fp32 scales.
@@ -49,7 +53,7 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = W.WORKLOADS[1].name
+DEFAULT_WORKLOAD = W.WORKLOADS[4].name
 METRIC = "µs/call and achieved HBM GB/s (fraction of B200 roofline) per (M,K)"
 FALLBACK_HBM_GBS = 6650.0
 FWD_SOURCES = ["swiglu_backward_int8_b200/csrc/fwd_kernel.cuh",
@@ -67,8 +71,14 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["sdq", "reference"], default="sdq")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--all-workloads", action="store_true",
-                    help="also time every workload and add a per_workload list")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per_workload list (every workload timed after the headline)")
+    ap.add_argument("--per-workload-ms", type=float, default=50.0,
+                    help="timed calls per workload: enough for about this many ms")
+    ap.add_argument("--traffic-probe", type=int, default=0, metavar="N",
+                    help="no timing: N rounds of (read a 512 MB buffer, one call, read it again) "
+                         "on one buffer set, for an ncu capture of the call's DRAM bytes including "
+                         "the write-backs of its outputs that the second read forces")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0 = min(steps, 50)")
@@ -136,7 +146,10 @@ def measured_peaks():
 
 def recorded_traffic(workload: str, sources=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current sources of that kernel (else None)."""
+    on the current sources of that kernel (else None): bytes read, bytes
+    written during the launch and, where recorded, the write-backs of its
+    outputs still dirty in L2 when it ends (forced out by a following read
+    of a buffer larger than L2)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -144,7 +157,7 @@ def recorded_traffic(workload: str, sources=None):
     for line in open(path):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload and parts[1] == sha:
-            return int(parts[2]) + int(parts[3])
+            return sum(int(v) for v in parts[2:5])
     return None
 
 
@@ -224,6 +237,18 @@ def dist_setup(args):
     return world, rank, local
 
 
+def workload_config(w: W.Workload, fmt=None, world: int = 1) -> dict:
+    """The line's `config`, the same in both arms: the workload, its formats,
+    the parallel layout and how L2 is kept out of the timing."""
+    fmt = fmt or PAGE_FORMAT
+    return {"workload": w.name, "M": w.M, "K": w.K, "group_size": w.group_size,
+            "io": "bf16 x, grad_y in; " + {"int8": "int8", "e4m3": "fp8 e4m3"}[fmt[0]]
+                  + " codes + " + fmt[1] + " scales out, y_s_t " + fmt[2],
+            "parallelism": f"replicas x{world} (no exchange)",
+            "l2": "inputs+outputs rotate over enough buffer sets to exceed 3x L2 "
+                  "(one set when a call's own bytes do)"}
+
+
 # ---------------------------------------------------------------- CPU oracle timing
 
 def time_oracle(w: W.Workload, x, gy, min_seconds=10.0, max_rows=None):
@@ -278,8 +303,9 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "K": w.K, "group_size": G,
-                   "step": "one 128-token group x all K channels (bounded sample)"},
+        "config": workload_config(w, None, args.gpus),
+        "step": "one 128-token group x all K channels of the workload (a bounded sample), "
+                "cycling through its token groups",
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"{args.steps} steps of one 128-token group x K={w.K}"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -428,7 +454,6 @@ def run_sdq(args):
     fmt = (args.codes, args.scales, args.y_scale_layout)
     ms, (t0, t1), nsets = measure_device(wr, x_np, gy_np, args.steps, args.warmup, device, fmt)
     clocks = sampler.summary(t0, t1)
-    sampler.stop()
     ms_max = parallel.max_over_ranks(ms, device)
     per_step_ms = ms_max / args.steps
     bytes_step = w.algorithmic_bytes(scale_bytes(fmt))
@@ -446,18 +471,30 @@ def run_sdq(args):
         e2e = e
 
     per = None
-    if args.all_workloads:
+    if not args.no_per_workload:
         per = []
+        cache = {w.name: (wr, x_np, gy_np)} if rank == 0 or world == 1 else {}
         for ow in W.WORKLOADS:
-            ox, og = W.make_inputs(ow)
-            osteps = max(20, min(args.steps, int(2e9 // max(1, ow.algorithmic_bytes())) + 20))
-            oms, _, ons = measure_device(ow, ox, og, osteps, args.warmup, device)
+            if ow.name in cache:
+                ow_r, ox, og = cache[ow.name]
+            else:
+                ow_r = W.Workload(ow.name, ow.M, ow.K, ow.sigma_x, ow.sigma_grad_y,
+                                  ow.seed + 1000 * rank, ow.group_size, ow.outlier_frac,
+                                  ow.outlier_mult, ow.zero_group_every)
+                ox, og = W.make_inputs(ow_r)
+            # enough calls for about per_workload_ms at a first guess of 4 TB/s (small
+            # workloads are launch-bound, so they run longer than that)
+            guess_us = max(5.0, ow.algorithmic_bytes() / 4e3 / 1e3)
+            osteps = int(min(10000, max(args.steps, args.per_workload_ms * 1e3 / guess_us)))
+            oms, (o0, o1), ons = measure_device(ow_r, ox, og, osteps, args.warmup, device)
             oms = parallel.max_over_ranks(oms, device)
             us = oms / osteps * 1e3
             gbs = ow.algorithmic_bytes() / (us * 1e-6) / 1e9
             per.append({"workload": ow.name, "M": ow.M, "K": ow.K, "us_per_call": us,
                         "GB_s": gbs, "frac_of_measured_hbm": gbs / peak, "frac_of_8TBs": gbs / 8000,
-                        "steps": osteps, "buffer_sets": ons})
+                        "algorithmic_bytes_per_launch": ow.algorithmic_bytes(),
+                        "steps": osteps, "buffer_sets": ons,
+                        "clocks_sm_mhz": sampler.summary(o0, o1).get("sm_mhz")})
             del ox, og
 
     per_fmt = None
@@ -498,9 +535,10 @@ def run_sdq(args):
         int8_gy = {"us_per_call": us, "GB_s": gbs, "frac_of_measured_hbm": gbs / peak,
                    "algorithmic_bytes_per_launch": qb, "format": format_name(PAGE_FORMAT)}
 
+    sampler.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0)
+        cpu = time_oracle(w, x_np, gy_np, min_seconds=10.0, max_rows=1024)
 
     if rank == 0:
         traffic = recorded_traffic(w.name) if fmt == PAGE_FORMAT else None
@@ -509,14 +547,12 @@ def run_sdq(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
             "us_per_call": per_step_ms * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name, "M": w.M, "K": w.K, "group_size": w.group_size,
-                       "io": "bf16 x, grad_y in; " + {"int8": "int8", "e4m3": "fp8 e4m3"}[fmt[0]]
-                             + " codes + " + fmt[1] + " scales out, y_s_t " + fmt[2],
-                       "parallelism": f"replicas x{world} (no exchange)",
-                       "l2": f"inputs+outputs rotate over {nsets} buffer sets (>= 3x L2)",
-                       "timing": "K calls replayed from CUDA graphs, CUDA events"},
+            "config": workload_config(w, fmt, world),
+            "buffer_sets": nsets,
+            "timing": "K calls replayed from CUDA graphs, CUDA events on the launching stream",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
+                         "frac_of_8TBs": achieved / 8000.0,
                          "traffic": traffic, "algorithmic_bytes_per_launch": bytes_step,
                          "kernel": "sdq::fuse_kernel"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
@@ -653,10 +689,45 @@ def run_fwd(args):
     return 0
 
 
+def run_traffic_probe(args):
+    """No timing: N rounds of (read a 512 MB buffer, one call of the op, read
+    the buffer again) on one GPU and one buffer set.  The first read leaves
+    only clean lines in L2, so the call's own DRAM writes are what ncu counts
+    for it; the second read evicts the outputs the call left dirty in L2, so
+    its DRAM writes are the call's remaining write-backs.  Capture with
+    ncu --cache-control none, kernels matching fuse_kernel|reduce_kernel,
+    skipping the first round (its first read also writes back the buffer's
+    initial fill)."""
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import swiglu_backward_int8_b200 as sdq  # fails loudly if the CUDA library is missing
+    w = pick_workload(args.workload)
+    x_np, gy_np = W.make_inputs(w)
+    xs, gs = _to_device_bf16(x_np, device), _to_device_bf16(gy_np, device)
+    outs = sdq.allocate_outputs(w.M, w.K, device)
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize(device)
+    for _ in range(args.traffic_probe):
+        flush.amax()
+        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs)
+        flush.amax()
+    torch.cuda.synchronize(device)
+    st = sdq.sdq_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {sdq.status_string(st)}")
+    print(json.dumps({"traffic_probe": w.name, "rounds": args.traffic_probe,
+                      "algorithmic_bytes_per_launch": w.algorithmic_bytes(),
+                      "kernel_sources_sha": kernel_sha()}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.traffic_probe:
+        return run_traffic_probe(args)
     if args.op == "swiglu_q8_1":
         return run_fwd(args)
     return run_sdq(args)

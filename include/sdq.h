@@ -24,12 +24,15 @@
  *   per group: amax = max |v|; all-zero group -> scale 1, q 0; otherwise
  *   scale = amax / 127 (fp32, correctly rounded) and
  *   q = round-half-even(v * (1/scale)) in [-127, 127];
- *   a tail token group (M % 128 != 0) is quantized over the tokens it holds.
+ *   a tail token group (M % 128 != 0) is quantized over the tokens it holds,
+ *   and likewise, when 128 does not divide K, the last channel group of each
+ *   half of [d_gate | d_up] over the K - 128 (Kg - 1) channels it holds
+ *   (Kg = ceil(K/128); groups never cross from d_gate into d_up).
  *
  * Output layouts (all row-major, contiguous):
  *   grad_input_q int8 [M, 2K]             columns 0..K-1 = d_gate, K..2K-1 = d_up
- *   grad_input_s fp32 [M, 2K/128]         column j < K/128: d_gate group j;
- *                                         column K/128 + j: d_up group j
+ *   grad_input_s fp32 [M, 2 Kg]           column j < Kg: d_gate group j;
+ *                                         column Kg + j: d_up group j
  *   y_q_t        int8 [K, M]              y transposed: y_q_t[k, m] quantizes y[m, k]
  *   y_s_t        fp32 [K, ceil(M/128)]    y_s_t[k, i]: scale of tokens 128i..128i+127
  * (for group_size 32 or 64 read that size for 128 in the scale shapes; the
@@ -41,6 +44,13 @@
  * asynchronous on the given stream (no implicit synchronization).  Calls on
  * different streams may run concurrently; concurrent calls must not share
  * output buffers.  Inputs and outputs must not overlap.
+ *
+ * Per-device state: the library sets up, once per device and process, the
+ * kernels' attributes, the copy streams and events of sdq_fuse_host, and
+ * the device address of sdq_fuse_host_noalloc's array.  All of it belongs
+ * to the device's primary context: after cudaDeviceReset (or anything else
+ * that destroys that context) the library must not be called again on that
+ * device in the same process.
  *
  * Errors: every entry point returns an sdq_status.  On a validation error
  * nothing is launched and nothing is written.  SDQ_ERR_CUDA means a CUDA
@@ -60,7 +70,7 @@ typedef enum sdq_status {
   SDQ_OK = 0,
   SDQ_ERR_NULL = 1,      /* a required pointer is NULL (with M > 0)                  */
   SDQ_ERR_GROUP = 2,     /* group_size not 32, 64 or 128 (host-buffer entries: 128)  */
-  SDQ_ERR_SHAPE = 3,     /* M < 0, K < 1, K % 128 != 0, or a size above the limits   */
+  SDQ_ERR_SHAPE = 3,     /* M < 0, K < 1, K % 16 != 0, or a size above the limits    */
   SDQ_ERR_ALIGN = 4,     /* x, grad_y, grad_input_q, y_q_t not 16-byte aligned, or a
                             scale pointer not 4-byte aligned                          */
   SDQ_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed (see sdq_last_cuda_error) */
@@ -77,6 +87,7 @@ typedef enum sdq_status {
 #define SDQ_GROUP_SIZE 128
 #define SDQ_MAX_M 2147483647LL
 #define SDQ_MAX_K 1048576LL
+#define SDQ_K_MULTIPLE 16      /* K must be a multiple of this (16-byte code rows)   */
 #define SDQ_MAX_LD (1LL << 36) /* largest leading dimension (tensor-map strides < 2^40 bytes) */
 #define SDQ_MAX_LD_ROWS (1LL << 24) /* largest ld of grad_input_q and grad_input_s     */
 
@@ -85,15 +96,16 @@ typedef enum sdq_status {
  *   x             device, bf16 [M, 2K], 16-byte aligned
  *   grad_y        device, bf16 [M, K], 16-byte aligned
  *   grad_input_q  device, int8 [M, 2K], 16-byte aligned      (written)
- *   grad_input_s  device, fp32 [M, 2K/128], 4-byte aligned   (written)
+ *   grad_input_s  device, fp32 [M, 2 ceil(K/128)], 4-byte aligned (written)
  *   y_q_t         device, int8 [K, M], 16-byte aligned       (written)
  *   y_s_t         device, fp32 [K, ceil(M/128)], 4-byte aligned (written)
  *   M             tokens (rows of x), 0 <= M <= SDQ_MAX_M; M == 0 is a no-op
- *   K             channels of gate/up, a positive multiple of 128, <= SDQ_MAX_K
+ *   K             channels of gate/up, a positive multiple of SDQ_K_MULTIPLE
+ *                 (16), <= SDQ_MAX_K
  *   group_size    128 (the page's), or 32 or 64: tokens per column group and
- *                 channels per row group; grad_input_s is then [M, 2K/group_size]
- *                 (d_up groups from column K/group_size on) and y_s_t
- *                 [K, ceil(M/group_size)]; K stays a multiple of 128
+ *                 channels per row group; grad_input_s is then
+ *                 [M, 2 ceil(K/group_size)] (d_up groups from column
+ *                 ceil(K/group_size) on) and y_s_t [K, ceil(M/group_size)]
  *   stream        a cudaStream_t (NULL = the legacy default stream)
  * Launches one persistent kernel on the current device.  Returns SDQ_OK once
  * the launch is enqueued.
@@ -164,7 +176,7 @@ int sdq_validate_format(const void* x, const void* grad_y, const void* grad_inpu
  *                      multiple of 8 (rows start on 16 bytes)
  *   grad_input_q       [M, 2K] codes; 16-byte aligned; ld a multiple of 16,
  *                      at most SDQ_MAX_LD_ROWS
- *   grad_input_s       [M, 2K/group_size] scales; 2K/group_size <= ld <=
+ *   grad_input_s       [M, 2 ceil(K/group_size)] scales; that many <= ld <=
  *                      SDQ_MAX_LD_ROWS
  *   y_q_t              [K, M] codes; 16-byte aligned; any ld >= M (a multiple
  *                      of 16 takes 16-byte stores, others byte stores)
@@ -204,8 +216,9 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
  * ("entry point" section) takes grad_y in bf16; this entry reads
  *   grad_y_q   device, INT8 codes [M, K]; 16-byte aligned; ld a multiple of
  *              16 (rows start on 16 bytes), K <= ld <= SDQ_MAX_LD
- *   grad_y_s   device, fp32 scales [M, K/128], one per token and 128
- *              consecutive channels; 4-byte aligned; K/128 <= ld <= SDQ_MAX_LD
+ *   grad_y_s   device, fp32 scales [M, ceil(K/128)], one per token and 128
+ *              consecutive channels (the last one of a row over what is
+ *              left); 4-byte aligned; ceil(K/128) <= ld <= SDQ_MAX_LD
  * and takes grad_y[m, k] = grad_y_q[m, k] * grad_y_s[m, k / 128], each
  * product rounded once to fp32; everything else (the optional y included)
  * as sdq_fuse_strided.  Statuses as sdq_fuse_strided, plus SDQ_ERR_NULL for a
@@ -308,7 +321,13 @@ size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows);
  *     returns SDQ_ERR_TOO_LARGE before any CUDA call.  M is unlimited.
  *   - Set-up: the first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  A failed lookup returns
+ *     SDQ_ERR_CUDA and is tried again by the next call.
+ *   - Host buffers: page-locked (cudaHostAlloc / cudaHostRegister) for the
+ *     copies to run asynchronously.  Pageable buffers give the same results,
+ *     but the CUDA runtime then copies through its own staging memory and
+ *     the device->host copies return only once they are done, so the call
+ *     blocks the host until the last chunk's kernel has run.
  *   - Sharing: all calls on a device share the one array, and it keeps the
  *     last call's contents (every byte a call reads is written by that same
  *     call first, so nothing needs clearing).  Calls that overlap on the GPU

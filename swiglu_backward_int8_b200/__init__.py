@@ -6,7 +6,7 @@ entry point and outputs sections).
                                 group_size=128)
 
 takes CUDA tensors x = [gate | up] (bf16 [M, 2K]) and grad_y (bf16 [M, K]) and
-writes, in place, grad_input_q (int8 [M, 2K]), grad_input_s (fp32 [M, 2K/128]),
+writes, in place, grad_input_q (int8 [M, 2K]), grad_input_s (fp32 [M, 2 ceil(K/128)]),
 y_q_t (int8 [K, M]) and y_s_t (fp32 [K, ceil(M/128)]).  PyTorch supplies only
 the device memory and the current stream; the work runs in libsdq.so.
 
@@ -37,11 +37,12 @@ __all__ = [
     "FMT_E4M3", "FMT_E8M0", "FMT_YS_MG_K", "sdq_fuse_host", "sdq_fuse_host_noalloc",
     "sdq_fuse_host_workspace_bytes", "sdq_validate",
     "sdq_device_status", "SdqError", "Status", "status_string", "last_cuda_error", "version",
-    "LIB_PATH", "GROUP_SIZE", "GROUP_SIZES",
+    "LIB_PATH", "GROUP_SIZE", "GROUP_SIZES", "K_MULTIPLE",
 ]
 
 GROUP_SIZE = 128
 GROUP_SIZES = (32, 64, 128)   # the kernel's tile (128 x 128) holds whole groups of these sizes
+K_MULTIPLE = 16               # K must be a multiple of this (a shorter last channel group otherwise)
 
 
 _E8M0_DTYPES = tuple(d for d in (torch.uint8, getattr(torch, "float8_e8m0fnu", None)) if d is not None)
@@ -63,7 +64,8 @@ def output_shapes(M: int, K: int, group_size: int = GROUP_SIZE, y_scale_layout: 
     """Shapes of (grad_input_q, grad_input_s, y_q_t, y_s_t)."""
     G = group_size
     Mg = (M + G - 1) // G
-    return (M, 2 * K), (M, 2 * (K // G)), (K, M), ((Mg, K) if y_scale_layout == "mg_k" else (K, Mg))
+    Kg = (K + G - 1) // G   # channel groups per half of [d_gate | d_up]; the last may be short
+    return (M, 2 * K), (M, 2 * Kg), (K, M), ((Mg, K) if y_scale_layout == "mg_k" else (K, Mg))
 
 
 def allocate_outputs(M: int, K: int, device, group_size: int = GROUP_SIZE, codes: str = "int8",
@@ -109,8 +111,9 @@ def _rows(name: str, t: torch.Tensor, shape, dtypes, want_cuda: bool, device) ->
 
 
 def _check_group(K: int, group_size: int, want_cuda: bool):
-    if group_size not in GROUP_SIZES or K % GROUP_SIZE:
-        raise ValueError(f"group_size must be one of {GROUP_SIZES} and K={K} a multiple of 128")
+    if group_size not in GROUP_SIZES or K % K_MULTIPLE or K < 1:
+        raise ValueError(f"group_size must be one of {GROUP_SIZES} and K={K} a positive multiple "
+                         f"of {K_MULTIPLE}")
     if not want_cuda and group_size != GROUP_SIZE:
         raise ValueError("the host-buffer entry points take group_size 128 only")
 
@@ -150,12 +153,13 @@ def _check_y(y, M, K, device):
 
 def _grad_y(grad_y, grad_y_s, M, K, device):
     """grad_y in bf16 [M, K], or INT8 codes [M, K] with fp32 scales
-    ``grad_y_s`` [M, K/128]: (its leading dimension, the scales' pointer or
+    ``grad_y_s`` [M, ceil(K/128)]: (its leading dimension, the scales' pointer or
     None, their leading dimension)."""
     if grad_y_s is None:
         return _rows("grad_y", grad_y, (M, K), (torch.bfloat16,), True, device), None, 0
     ld_q = _rows("grad_y", grad_y, (M, K), (torch.int8,), True, device)
-    ld_s = _rows("grad_y_s", grad_y_s, (M, K // GROUP_SIZE), (torch.float32,), True, device)
+    ld_s = _rows("grad_y_s", grad_y_s, (M, (K + GROUP_SIZE - 1) // GROUP_SIZE), (torch.float32,), True,
+                 device)
     return ld_q, grad_y_s.data_ptr(), ld_s
 
 
@@ -189,7 +193,7 @@ def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_inpu
     tensor is 2-D row-major; rows may be padded (a slice of a wider buffer):
     the library takes each tensor's row stride.  ``y`` (bf16 [M, K], optional)
     also receives the recomputed y itself, the values y_q_t quantizes.  With
-    ``grad_y_s`` (fp32 [M, K/128]) grad_y is INT8 codes [M, K] standing for
+    ``grad_y_s`` (fp32 [M, ceil(K/128)]) grad_y is INT8 codes [M, K] standing for
     grad_y * grad_y_s[m, k // 128] (grad_y handed over already quantized).
     Raises ValueError on bad arguments and SdqError on a library status."""
     outs = (grad_input_q, grad_input_s, y_q_t, y_s_t)

@@ -194,7 +194,7 @@ Arrays packed(const void* x, const void* gy, void* giq, void* gis, void* yqt, vo
   a.giq = giq;
   a.ld_giq = 2 * K;
   a.gis = gis;
-  a.ld_gis = 2 * K / gsz;
+  a.ld_gis = 2 * ((K + gsz - 1) / gsz);
   a.yqt = yqt;
   a.ld_yqt = M;
   a.yst = yst;
@@ -222,9 +222,9 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   p.yst = a.yst;
   p.M = M;
   p.K = static_cast<int32_t>(K);
-  p.Kg = static_cast<int32_t>(K / sdq::kG);
+  p.Kg = static_cast<int32_t>((K + sdq::kG - 1) / sdq::kG);
   p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
-  p.gis_cols = static_cast<int32_t>(2 * K / group_size);
+  p.gis_cols = static_cast<int32_t>(2 * ((K + group_size - 1) / group_size));
   p.ld_giq = static_cast<int32_t>(a.ld_giq);
   p.ld_gis = static_cast<int32_t>(a.ld_gis);
   p.ld_yqt = a.ld_yqt;
@@ -265,7 +265,7 @@ struct ChunkLayout {
 };
 
 ChunkLayout chunk_layout(int64_t CR, int64_t K) {
-  const int64_t Kg = K / sdq::kG;
+  const int64_t Kg = (K + sdq::kG - 1) / sdq::kG;
   ChunkLayout L;
   size_t off = 0;
   L.x = off;   off += align256(size_t(CR) * 2 * K * 2);
@@ -300,7 +300,7 @@ const char* sdq_status_string(int status) {
     case SDQ_OK: return "SDQ_OK";
     case SDQ_ERR_NULL: return "SDQ_ERR_NULL: a required pointer is NULL";
     case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 32, 64 or 128 (128 for the host-buffer entry points)";
-    case SDQ_ERR_SHAPE: return "SDQ_ERR_SHAPE: need M >= 0 and K a positive multiple of 128 within the size limits";
+    case SDQ_ERR_SHAPE: return "SDQ_ERR_SHAPE: need M >= 0 and K a positive multiple of 16 within the size limits";
     case SDQ_ERR_ALIGN: return "SDQ_ERR_ALIGN: x, grad_y, grad_input_q, y_q_t need 16-byte and scales 4-byte alignment";
     case SDQ_ERR_CUDA: return "SDQ_ERR_CUDA: a CUDA call failed (see sdq_last_cuda_error)";
     case SDQ_ERR_TIMEOUT: return "SDQ_ERR_TIMEOUT: a device-side wait ran past its limit";
@@ -321,9 +321,10 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
   if (format & ~static_cast<uint32_t>(SDQ_FMT_E4M3 | SDQ_FMT_E8M0 | SDQ_FMT_YS_MG_K))
     return SDQ_ERR_FORMAT;
   if (!group_size_supported(group_size)) return SDQ_ERR_GROUP;
-  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
+  if (M < 0 || K < 1 || K % SDQ_K_MULTIPLE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
     return SDQ_ERR_SHAPE;
-  const int64_t tiles = ((M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE) * (K / SDQ_GROUP_SIZE);
+  const int64_t tiles = ((M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE) *
+                        ((K + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE);
   if (tiles > INT32_MAX) return SDQ_ERR_SHAPE;
   if (M == 0) return SDQ_OK;
   if (!gate || !up || !grad_y || !grad_input_q || !grad_input_s || !y_q_t || !y_s_t)
@@ -331,7 +332,7 @@ int sdq_validate_strided(const void* gate, int64_t ld_gate, const void* up, int6
   const int64_t groups_m = (M + group_size - 1) / group_size;
   const int64_t need_yst = (format & SDQ_FMT_YS_MG_K) ? K : groups_m;
   const int64_t lds[7] = {ld_gate, ld_up, ld_grad_y, ld_grad_input_q, ld_grad_input_s, ld_y_q_t, ld_y_s_t};
-  const int64_t need[7] = {K, K, K, 2 * K, 2 * K / group_size, M, need_yst};
+  const int64_t need[7] = {K, K, K, 2 * K, 2 * ((K + group_size - 1) / group_size), M, need_yst};
   for (int k = 0; k < 7; ++k)
     if (lds[k] < need[k] || lds[k] > SDQ_MAX_LD) return SDQ_ERR_STRIDE;
   if (ld_grad_input_q > SDQ_MAX_LD_ROWS || ld_grad_input_s > SDQ_MAX_LD_ROWS) return SDQ_ERR_STRIDE;
@@ -403,7 +404,8 @@ int sdq_validate_int8_grad_y(const void* gate, int64_t ld_gate, const void* up, 
                                       ld_y_q_t, y_s_t, ld_y_s_t, y, ld_y, M, K, group_size, format);
   if (st != SDQ_OK || M == 0) return st;
   if (!grad_y_s) return SDQ_ERR_NULL;
-  if (ld_grad_y_s < K / SDQ_GROUP_SIZE || ld_grad_y_s > SDQ_MAX_LD) return SDQ_ERR_STRIDE;
+  if (ld_grad_y_s < (K + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE || ld_grad_y_s > SDQ_MAX_LD)
+    return SDQ_ERR_STRIDE;
   // code rows start on 16 bytes (tensor-map stride); scales are fp32
   if ((ld_grad_y_q & 15) || (reinterpret_cast<uintptr_t>(grad_y_s) & 3u)) return SDQ_ERR_ALIGN;
   return SDQ_OK;
@@ -433,7 +435,7 @@ int sdq_fuse(const void* x, const void* grad_y, int8_t* grad_input_q, float* gra
 }
 
 size_t sdq_fuse_host_workspace_bytes(int64_t M, int64_t K, int64_t chunk_rows) {
-  if (M < 1 || K < 1 || K % SDQ_GROUP_SIZE != 0 || K > SDQ_MAX_K || M > SDQ_MAX_M) return 0;
+  if (M < 1 || K < 1 || K % SDQ_K_MULTIPLE != 0 || K > SDQ_MAX_K || M > SDQ_MAX_M) return 0;
   if (chunk_rows < 0 || chunk_rows % SDQ_GROUP_SIZE != 0) return 0;
   const int64_t CR = chunk_rows ? chunk_rows : choose_chunk_rows(M, K);
   return 2 * chunk_layout(CR, K).total;
@@ -443,7 +445,7 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
                   int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K, int32_t group_size,
                   void* workspace, size_t workspace_bytes, int64_t chunk_rows, void* stream) {
   if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
-  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K ||
+  if (M < 0 || K < 1 || K % SDQ_K_MULTIPLE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K ||
       chunk_rows < 0 || chunk_rows % SDQ_GROUP_SIZE != 0)
     return SDQ_ERR_SHAPE;
   if (M == 0) return SDQ_OK;
@@ -469,7 +471,7 @@ int sdq_fuse_host(const void* x, const void* grad_y, int8_t* grad_input_q, float
     d->pipe_ready = true;
   }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const int64_t Kg = K / SDQ_GROUP_SIZE;
+  const int64_t Kg = (K + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
   const int64_t Mg = (M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
   const auto* xh = static_cast<const uint8_t*>(x);
   const auto* gh = static_cast<const uint8_t*>(grad_y);
@@ -534,9 +536,11 @@ namespace {
 // the device address looked up per device below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SDQ_NOALLOC_SCRATCH_BYTES];
 
+// The array's device address per device, looked up by the first call that
+// succeeds in doing so (a failed lookup is not remembered: the next call
+// tries again).
 struct NoallocDevice {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
+  std::mutex mu;
   uint8_t* ptr = nullptr;
 };
 NoallocDevice g_noalloc[kMaxDevices];
@@ -558,7 +562,7 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
                           float* grad_input_s, int8_t* y_q_t, float* y_s_t, int64_t M, int64_t K,
                           int32_t group_size, void* stream) {
   if (group_size != SDQ_GROUP_SIZE) return SDQ_ERR_GROUP;
-  if (M < 0 || K < 1 || K % SDQ_GROUP_SIZE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
+  if (M < 0 || K < 1 || K % SDQ_K_MULTIPLE != 0 || M > SDQ_MAX_M || K > SDQ_MAX_K)
     return SDQ_ERR_SHAPE;
   if (K > SDQ_NOALLOC_MAX_K) return SDQ_ERR_TOO_LARGE;
   if (M == 0) return SDQ_OK;
@@ -573,14 +577,19 @@ int sdq_fuse_host_noalloc(const void* x, const void* grad_y, int8_t* grad_input_
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
   NoallocDevice& nd = g_noalloc[dev];
-  std::call_once(nd.once, [&nd] {
-    nd.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&nd.ptr), g_noalloc_scratch);
-  });
-  if (nd.err != cudaSuccess) return cuda_fail(nd.err);
-  uint8_t* base = nd.ptr;
+  uint8_t* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(nd.mu);
+    if (!nd.ptr) {
+      void* p = nullptr;
+      if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return cuda_fail(e);
+      nd.ptr = static_cast<uint8_t*>(p);
+    }
+    base = nd.ptr;
+  }
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const int64_t Kg = K / SDQ_GROUP_SIZE;
+  const int64_t Kg = (K + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
   const int64_t Mg = (M + SDQ_GROUP_SIZE - 1) / SDQ_GROUP_SIZE;
   const auto* xh = static_cast<const uint8_t*>(x);
   const auto* gh = static_cast<const uint8_t*>(grad_y);

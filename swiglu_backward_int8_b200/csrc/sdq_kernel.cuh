@@ -92,8 +92,8 @@ struct Params {
   void* yst;     // [K, Mg] or [Mg, K], fp32 or E8M0 bytes
   int64_t M;
   int32_t K;
-  int32_t Kg;        // 128-channel tiles per row
-  int32_t gis_cols;  // 2K / group size: columns of grad_input_s (d_up groups from gis_cols/2)
+  int32_t Kg;        // 128-channel tiles per row (the last one may be partial: K % 128 != 0)
+  int32_t gis_cols;  // 2 ceil(K / group size): columns of grad_input_s (d_up groups from gis_cols/2)
   uint8_t* y;        // optional bf16 y [M, K] (kernels built with kY)
   int64_t ld_y;
   const float* gys;  // INT8 grad_y's scales [M, K/128] (kernels built with kQdy)
@@ -424,12 +424,13 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   group_scale<kE4M3, kE8M0>(m & 0xFFFFu, tab, s_lo, i_lo);
   group_scale<kE4M3, kE8M0>(m >> 16, tab, s_hi, i_hi);
   const int ch = j * kG + 2 * cp;
+  const bool ch_ok = ch < p.K;     // a partial channel tile's missing channels are zeros, not stored
   // the first two threads of each token group store its low / high channel
   // scale, for the groups that hold a token (a tail tile's later groups don't)
   constexpr int kTpg = kGS / 16;   // threads per token group
   const int gk = kc & (kTpg - 1);
   const int tg = kc / kTpg;        // token group within the tile
-  if (gk < 2 && tg * kGS < valid) {
+  if (gk < 2 && tg * kGS < valid && ch_ok) {
     const int64_t grp = int64_t(i) * (kG / kGS) + tg;
     store_scale<kE8M0>(p.yst, kYsMgK ? grp * p.ld_yst + ch + gk : int64_t(ch + gk) * p.ld_yst + grp,
                        gk ? s_hi : s_lo);
@@ -445,7 +446,7 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
                              lo, hi);
   }
   const int tok = 16 * kc;
-  if (tok < valid) {
+  if (tok < valid && ch_ok) {
     const int nb = min(16, valid - tok);
     int8_t* dst = p.yqt + int64_t(ch) * p.ld_yqt + row0 + tok;
     store_codes(dst, lo, nb, p.yqt_vec16 != 0);
@@ -528,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tile_ij(t, p.Mg, Kg, i, j);
     const int64_t row0 = int64_t(i) * kG;
     const int valid = static_cast<int>(M - row0 < kG ? M - row0 : int64_t(kG));
+    const int cvalid = min(kG, K - j * kG);   // channels of this tile (K % 128 != 0: fewer in the last)
     const int yb = k % kYBuf;   // y buffer of this tile; tile t completes phase t / kYBuf of its barriers
     uint8_t* yt = s.ytile[yb];
     // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
@@ -612,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int yr = sub * kStageRows + srow;
         if (yr < valid) {
           int8_t* yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + yr) * p.ld_y + int64_t(j) * kG);
-          st_cs_v4(yg + ca * 16, make_uint4(yv[0], yv[1], yv[2], yv[3]));
-          st_cs_v4(yg + cb * 16, make_uint4(yv[4], yv[5], yv[6], yv[7]));
+          if (ca * 8 < cvalid) st_cs_v4(yg + ca * 16, make_uint4(yv[0], yv[1], yv[2], yv[3]));
+          if (cb * 8 < cvalid) st_cs_v4(yg + cb * 16, make_uint4(yv[4], yv[5], yv[6], yv[7]));
         }
       }
 
@@ -638,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         constexpr int kLpg = kGS / 16;   // lanes per channel group
         const int gl = cq & (kLpg - 1);
-        if (gl < 2 && rbase + rr < valid)
+        if (gl < 2 && rbase + rr < valid && (cq / kLpg) * kGS < cvalid)
           store_scale<kE8M0>(p.gis, gis_t + (rbase + rr) * p.ld_gis + cq / kLpg +
                                         gl * (p.gis_cols >> 1),
                              gl ? su : sg);
@@ -656,10 +658,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ou = quant16<kE4M3, false>(dup, iu, su);
         }
         int8_t* dst = giq_t + r * p.ld_giq;
-        st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
-        st_cs_v2(dst + cb * 8, make_uint2(og.z, og.w));
-        st_cs_v2(dst + K + ca * 8, make_uint2(ou.x, ou.y));
-        st_cs_v2(dst + K + cb * 8, make_uint2(ou.z, ou.w));
+        if (ca * 8 < cvalid) {
+          st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
+          st_cs_v2(dst + K + ca * 8, make_uint2(ou.x, ou.y));
+        }
+        if (cb * 8 < cvalid) {
+          st_cs_v2(dst + cb * 8, make_uint2(og.z, og.w));
+          st_cs_v2(dst + K + cb * 8, make_uint2(ou.z, ou.w));
+        }
       }
     }
     if (!ok) break;

@@ -54,7 +54,10 @@ A = 1 << 20  # a 16-byte-aligned fake address: validation never dereferences
     (dict(group_size=32), 0),
     (dict(group_size=96), 2),
     (dict(group_size=256), 2),
-    (dict(group_size=64, K=192), 3),      # the tile stays 128 channels wide
+    (dict(group_size=64, K=192), 0),      # a shorter last channel tile
+    (dict(K=144), 0),                     # 128 + 16: the last channel group holds 16
+    (dict(K=16), 0),
+    (dict(K=136), 3),                     # K must be a multiple of 16
     (dict(K=100), 3),
     (dict(K=0), 3),
     (dict(M=-1), 3),

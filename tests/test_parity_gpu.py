@@ -163,42 +163,24 @@ def _tiles_to_sample(Mg, Kg, n, seed):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("idx", [4, 2])
-def test_full_size_sampled_tiles_and_invariants(idx):
-    """Full-size workloads in the bench's launch configuration: sampled tiles
-    against the oracle (each tile holds whole groups on both axes), and
-    properties that hold at any size checked over every element."""
-    import swiglu_backward_int8_b200 as sdq
-    w = W.WORKLOADS[idx]
-    x, gy = W.make_inputs(w)
+def test_largest_workload_in_full_and_invariants():
+    """M=16384 K=7168 (the bandwidth-roofline workload, 1.07 GB a call) in the
+    bench's launch configuration: every element of all four outputs against
+    the oracle on the whole op (about 8 s of one CPU core), every element
+    written and nothing outside, and properties that hold at any size: each
+    group's largest |q| is 127 unless the group is all zero (scale 1, q 0)."""
+    w = W.WORKLOADS[4]
     M, K, G = w.M, w.K, 128
-    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
-    outs = sdq.allocate_outputs(M, K, "cuda")
-    for t in outs:
-        t.fill_(U.SENTINEL_Q if t.dtype == torch.int8 else float("nan"))
-    sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *outs)
-    torch.cuda.synchronize()
-    assert sdq.sdq_device_status() == 0
-    giq, gis, yqt, yst = outs
-    # every element written; scales finite and positive
-    assert not (giq == U.SENTINEL_Q).any() and not (yqt == U.SENTINEL_Q).any()
-    assert torch.isfinite(gis).all() and (gis > 0).all()
-    assert torch.isfinite(yst).all() and (yst > 0).all()
-    # each group's largest |q| is 127 unless the group is all zero (scale 1, q 0)
-    rmax = giq.view(M, 2 * w.Kg, G).abs().amax(dim=2)
+    x, gy = W.make_inputs(w)
+    got = U.run_cuda(x, gy)          # guard bytes, sentinels, device status
+    giq, gis, yqt, yst = got
+    assert (gis > 0).all() and (yst > 0).all()
+    rmax = np.abs(giq.reshape(M, 2 * w.Kg, G).astype(np.int16)).max(axis=2)
     assert ((rmax == 127) | ((rmax == 0) & (gis == 1))).all()
-    cmax = yqt.view(K, M // G, G).abs().amax(dim=2)
+    cmax = np.abs(yqt.reshape(K, M // G, G).astype(np.int16)).max(axis=2)
     assert ((cmax == 127) | ((cmax == 0) & (yst == 1))).all()
-    host = [t.cpu().numpy() for t in outs]
-    n_diff = n_all = 0
-    for (i, j) in _tiles_to_sample(w.Mg, w.Kg, 40, seed=idx):
-        ref = U.oracle_tile(x, gy, i, j)
-        got = U.tile_of(host, M, K, i, j)
-        st = U.compare(got, ref, f"{w.name} tile ({i},{j})", max_frac=1.0)   # bound over the sample
-        n_diff += st["grad_input_q"]["n_diff"] + st["y_q_t"]["n_diff"]
-        n_all += ref[0].size + ref[2].size
-    assert n_diff <= U.INT8_MAX_FRAC * n_all, f"{n_diff} of {n_all} sampled codes differ"
-    _STATS[w.name + " (40 sampled tiles)"] = {"int8_n_diff": n_diff, "sampled_codes": n_all}
+    ref = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, w.group_size)
+    _STATS[w.name] = U.compare(got, ref, w.name)
 
 
 def test_scales_exact_over_the_whole_exponent_range():
