@@ -35,9 +35,9 @@
  *                                         column Kg + j: d_up group j
  *   y_q_t        int8 [K, M]              y transposed: y_q_t[k, m] quantizes y[m, k]
  *   y_s_t        fp32 [K, ceil(M/128)]    y_s_t[k, i]: scale of tokens 128i..128i+127
- * (for group_size 32 or 64 read that size for 128 in the scale shapes; the
- * group_size argument is the page's, the smaller groups its other values
- * that a 128 x 128 tile holds whole.)
+ * (for group_size 32, 64 or 256 read that size for 128 in the scale shapes;
+ * the group_size argument is the page's: 32 and 64 are groups a 128 x 128
+ * tile holds whole, 256 runs a kernel with 256 x 256 units.)
  *
  * Threading and ownership: the caller owns every buffer.  The device entry
  * point allocates nothing, keeps no pointer after it returns, and is
@@ -69,7 +69,7 @@ extern "C" {
 typedef enum sdq_status {
   SDQ_OK = 0,
   SDQ_ERR_NULL = 1,      /* a required pointer is NULL (with M > 0)                  */
-  SDQ_ERR_GROUP = 2,     /* group_size not 32, 64 or 128 (host-buffer entries: 128)  */
+  SDQ_ERR_GROUP = 2,     /* group_size not 32, 64, 128 or 256 (host-buffer entries: 128) */
   SDQ_ERR_SHAPE = 3,     /* M < 0, K < 1, K % 16 != 0, or a size above the limits    */
   SDQ_ERR_ALIGN = 4,     /* x, grad_y, grad_input_q, y_q_t not 16-byte aligned, or a
                             scale pointer not 4-byte aligned                          */
@@ -102,8 +102,8 @@ typedef enum sdq_status {
  *   M             tokens (rows of x), 0 <= M <= SDQ_MAX_M; M == 0 is a no-op
  *   K             channels of gate/up, a positive multiple of SDQ_K_MULTIPLE
  *                 (16), <= SDQ_MAX_K
- *   group_size    128 (the page's), or 32 or 64: tokens per column group and
- *                 channels per row group; grad_input_s is then
+ *   group_size    128 (the page's), or 32, 64 or 256: tokens per column group
+ *                 and channels per row group; grad_input_s is then
  *                 [M, 2 ceil(K/group_size)] (d_up groups from column
  *                 ceil(K/group_size) on) and y_s_t [K, ceil(M/group_size)]
  *   stream        a cudaStream_t (NULL = the legacy default stream)

@@ -41,7 +41,7 @@ __all__ = [
 ]
 
 GROUP_SIZE = 128
-GROUP_SIZES = (32, 64, 128)   # the kernel's tile (128 x 128) holds whole groups of these sizes
+GROUP_SIZES = (32, 64, 128, 256)   # 128 x 128 tiles hold whole groups of 32..128; 256: 256 x 256 units
 K_MULTIPLE = 16               # K must be a multiple of this (a shorter last channel group otherwise)
 
 
@@ -189,7 +189,7 @@ def silu_dot_fwd_bwd_quant_fuse(x: torch.Tensor, grad_y: torch.Tensor, grad_inpu
     current CUDA stream of x's device.  The code format ("int8" or "e4m3")
     and the scale format ("fp32" or "e8m0") follow the dtypes of
     grad_input_q and grad_input_s unless given; ``y_scale_layout`` is "k_mg"
-    (y_s_t [K, ceil(M/G)]) or "mg_k"; ``group_size`` is 128, 64 or 32.  Every
+    (y_s_t [K, ceil(M/G)]) or "mg_k"; ``group_size`` is 128, 64, 32 or 256.  Every
     tensor is 2-D row-major; rows may be padded (a slice of a wider buffer):
     the library takes each tensor's row stride.  ``y`` (bf16 [M, K], optional)
     also receives the recomputed y itself, the values y_q_t quantizes.  With

@@ -12,6 +12,7 @@
 
 #include "sdq.h"
 #include "sdq_kernel.cuh"
+#include "sdq_kernel256.cuh"
 
 namespace {
 
@@ -24,12 +25,14 @@ constexpr int kStages = SDQ_STAGES;
 
 constexpr int kMaxDevices = 64;
 
-// One kernel per group size (32, 64, 128), output format (SDQ_FMT_* bits
-// 0..2), whether bf16 y is written too, and whether grad_y comes as INT8
-// codes with scales.
+// One kernel per group size (32, 64, 128 in the 128 x 128-tile kernel; 256
+// in the 256 x 256-unit kernel), output format (SDQ_FMT_* bits 0..2),
+// whether bf16 y is written too, and whether grad_y comes as INT8 codes with
+// scales.
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const sdq::Params);
 constexpr int kFormats = 8;
-constexpr int kKernels = 2 * 2 * 3 * kFormats;
+constexpr int kGroupSizes = 4;
+constexpr int kKernels = 2 * 2 * kGroupSizes * kFormats;
 
 template <int G, bool kY, bool kQ>
 constexpr KernelFn kernel_of(int f) {
@@ -46,15 +49,30 @@ constexpr KernelFn kernel_of(int f) {
 }
 
 template <bool kY, bool kQ>
-KernelFn kernel_of_group(int g, int f) {
-  return g == 0 ? kernel_of<32, kY, kQ>(f) : g == 1 ? kernel_of<64, kY, kQ>(f) : kernel_of<128, kY, kQ>(f);
+constexpr KernelFn kernel256_of(int f) {
+  switch (f) {
+    case 0: return sdq::fuse256_kernel<kStages, false, false, false, kY, kQ>;
+    case 1: return sdq::fuse256_kernel<kStages, true, false, false, kY, kQ>;
+    case 2: return sdq::fuse256_kernel<kStages, false, true, false, kY, kQ>;
+    case 3: return sdq::fuse256_kernel<kStages, true, true, false, kY, kQ>;
+    case 4: return sdq::fuse256_kernel<kStages, false, false, true, kY, kQ>;
+    case 5: return sdq::fuse256_kernel<kStages, true, false, true, kY, kQ>;
+    case 6: return sdq::fuse256_kernel<kStages, false, true, true, kY, kQ>;
+    default: return sdq::fuse256_kernel<kStages, true, true, true, kY, kQ>;
+  }
 }
 
-// Kernel number n = 48 * (INT8 grad_y) + 24 * (y written) + 8 * (0, 1, 2 for
-// group size 32, 64, 128) + format bits.
+template <bool kY, bool kQ>
+KernelFn kernel_of_group(int g, int f) {
+  return g == 0 ? kernel_of<32, kY, kQ>(f) : g == 1 ? kernel_of<64, kY, kQ>(f)
+       : g == 2 ? kernel_of<128, kY, kQ>(f) : kernel256_of<kY, kQ>(f);
+}
+
+// Kernel number n = 32 * (2 * INT8 grad_y + y written) + 8 * (0, 1, 2, 3 for
+// group size 32, 64, 128, 256) + format bits.
 KernelFn kernel_at(int n) {
-  const int v = n / (3 * kFormats);   // 0..3: (y, INT8 grad_y) bits
-  const int g = (n % (3 * kFormats)) / kFormats, f = n % kFormats;
+  const int v = n / (kGroupSizes * kFormats);   // 0..3: (y, INT8 grad_y) bits
+  const int g = (n % (kGroupSizes * kFormats)) / kFormats, f = n % kFormats;
   switch (v) {
     case 0: return kernel_of_group<false, false>(g, f);
     case 1: return kernel_of_group<true, false>(g, f);
@@ -63,13 +81,23 @@ KernelFn kernel_at(int n) {
   }
 }
 
+bool is_group256(int n) { return (n % (kGroupSizes * kFormats)) / kFormats == 3; }
+
+int group_index(int32_t group_size) {
+  return group_size == 32 ? 0 : group_size == 64 ? 1 : group_size == 128 ? 2 : 3;
+}
+
 KernelFn kernel_for(int32_t group_size, uint32_t format, bool y, bool qdy) {
-  const int gi = group_size == 32 ? 0 : group_size == 64 ? 1 : 2;
-  return kernel_at(((qdy ? 2 : 0) + (y ? 1 : 0)) * 3 * kFormats + gi * kFormats +
+  return kernel_at(((qdy ? 2 : 0) + (y ? 1 : 0)) * kGroupSizes * kFormats + group_index(group_size) * kFormats +
                    static_cast<int>(format & (kFormats - 1)));
 }
 
-bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE; }
+// Dynamic shared memory of the kernel for a group size.
+size_t smem_for(int32_t group_size) {
+  return group_size == 256 ? sdq::smem_bytes256<kStages>() : sdq::smem_bytes<kStages>();
+}
+
+bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE || g == 256; }
 thread_local int t_last_cuda_error = 0;
 
 int cuda_fail(cudaError_t e) {
@@ -132,13 +160,13 @@ int current_device(DeviceState** out) {
     d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     for (int n = 0; n < kKernels; ++n) {
       const auto kernel = kernel_at(n);
+      const size_t smem = is_group256(n) ? sdq::smem_bytes256<kStages>() : sdq::smem_bytes<kStages>();
       if (d.init_err == cudaSuccess)
         d.init_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(sdq::smem_bytes<kStages>()));
+                                          static_cast<int>(smem));
       int blocks = 0;
       if (d.init_err == cudaSuccess)
-        d.init_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel, sdq::kThreads,
-                                                                   sdq::smem_bytes<kStages>());
+        d.init_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel, sdq::kThreads, smem);
       if (d.init_err == cudaSuccess && blocks < 1) d.init_err = cudaErrorLaunchOutOfResources;
     }
   });
@@ -150,12 +178,14 @@ int current_device(DeviceState** out) {
 // A [rows, inner] row-major array of bf16 (or, with `bytes`, 8-bit codes)
 // read in boxes of 64 rows x 128 elements.
 int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-             uint64_t row_bytes, bool bytes = false) {
+             uint64_t row_bytes, bool bytes = false, bool group256 = false) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(sdq::kG), static_cast<cuuint32_t>(sdq::kStageRows)};
+  // boxes of 64 rows x 128 elements, or 32 rows x 256 for the 256-group kernel
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(group256 ? sdq::kG2 : sdq::kG),
+                             static_cast<cuuint32_t>(group256 ? sdq::kStageRows2 : sdq::kStageRows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                   const_cast<void*>(base), dims, strides,
@@ -210,11 +240,13 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   DeviceState* d = nullptr;
   int st = current_device(&d);
   if (st != SDQ_OK) return st;
+  const bool g256 = group_size == 256;
+  const int64_t unit = g256 ? sdq::kG2 : sdq::kG;   // tile / unit edge
   CUtensorMap mgate, mup, mdy;
-  if ((st = make_map(&mgate, a.gate, K, M, 2 * a.ld_gate)) != SDQ_OK) return st;
-  if ((st = make_map(&mup, a.up, K, M, 2 * a.ld_up)) != SDQ_OK) return st;
+  if ((st = make_map(&mgate, a.gate, K, M, 2 * a.ld_gate, false, g256)) != SDQ_OK) return st;
+  if ((st = make_map(&mup, a.up, K, M, 2 * a.ld_up, false, g256)) != SDQ_OK) return st;
   const bool qdy = a.gys != nullptr;
-  if ((st = make_map(&mdy, a.gy, K, M, (qdy ? 1 : 2) * a.ld_gy, qdy)) != SDQ_OK) return st;
+  if ((st = make_map(&mdy, a.gy, K, M, (qdy ? 1 : 2) * a.ld_gy, qdy, g256)) != SDQ_OK) return st;
   sdq::Params p;
   p.giq = static_cast<int8_t*>(a.giq);
   p.gis = a.gis;
@@ -222,8 +254,8 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   p.yst = a.yst;
   p.M = M;
   p.K = static_cast<int32_t>(K);
-  p.Kg = static_cast<int32_t>((K + sdq::kG - 1) / sdq::kG);
-  p.Mg = static_cast<int32_t>((M + sdq::kG - 1) / sdq::kG);
+  p.Kg = static_cast<int32_t>((K + unit - 1) / unit);
+  p.Mg = static_cast<int32_t>((M + unit - 1) / unit);
   p.gis_cols = static_cast<int32_t>(2 * ((K + group_size - 1) / group_size));
   p.ld_giq = static_cast<int32_t>(a.ld_giq);
   p.ld_gis = static_cast<int32_t>(a.ld_gis);
@@ -244,7 +276,7 @@ int launch(const Arrays& a, int64_t M, int64_t K, int32_t group_size, uint32_t f
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(sdq::kThreads);
-  cfg.dynamicSmemBytes = sdq::smem_bytes<kStages>();
+  cfg.dynamicSmemBytes = smem_for(group_size);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -299,7 +331,7 @@ const char* sdq_status_string(int status) {
   switch (status) {
     case SDQ_OK: return "SDQ_OK";
     case SDQ_ERR_NULL: return "SDQ_ERR_NULL: a required pointer is NULL";
-    case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 32, 64 or 128 (128 for the host-buffer entry points)";
+    case SDQ_ERR_GROUP: return "SDQ_ERR_GROUP: group_size must be 32, 64, 128 or 256 (128 for the host-buffer entry points)";
     case SDQ_ERR_SHAPE: return "SDQ_ERR_SHAPE: need M >= 0 and K a positive multiple of 16 within the size limits";
     case SDQ_ERR_ALIGN: return "SDQ_ERR_ALIGN: x, grad_y, grad_input_q, y_q_t need 16-byte and scales 4-byte alignment";
     case SDQ_ERR_CUDA: return "SDQ_ERR_CUDA: a CUDA call failed (see sdq_last_cuda_error)";

@@ -53,7 +53,8 @@ A = 1 << 20  # a 16-byte-aligned fake address: validation never dereferences
     (dict(group_size=64), 0),
     (dict(group_size=32), 0),
     (dict(group_size=96), 2),
-    (dict(group_size=256), 2),
+    (dict(group_size=256), 0),            # 256 x 256 units
+    (dict(group_size=512), 2),
     (dict(group_size=64, K=192), 0),      # a shorter last channel tile
     (dict(K=144), 0),                     # 128 + 16: the last channel group holds 16
     (dict(K=16), 0),

@@ -1,10 +1,13 @@
-"""CUDA path vs the oracle with quantization groups of 32 and 64 (the page's
-group_size argument; 128 is covered by the other parity tests), in the page's
-output format and the others, on the same seeded inputs.
+"""CUDA path vs the oracle with quantization groups of 32, 64 and 256 (the
+page's group_size argument; 128 is covered by the other parity tests), in the
+page's output format and the others, on the same seeded inputs.
 
 A 128 x 128 tile holds 16 (4) groups of 32 (64) on each axis; token groups
 wholly past M in a tail tile are not written, which the guarded, prefilled
-outputs check.  Tolerances: tests/gpu_util.py (compare_fmt).
+outputs check.  Groups of 256 run the kernel with 256 x 256 units: with
+K % 256 != 0 the last unit holds a shorter channel group (K = 128, 384 and
+1408 below), with M % 256 != 0 a tail token group.  Tolerances:
+tests/gpu_util.py (compare_fmt).
 """
 from __future__ import annotations
 
@@ -30,7 +33,7 @@ def _check(x, gy, G, fmt, where):
 
 
 @pytest.mark.parametrize("fmt", ALL_FORMATS, ids=FMT_IDS)
-@pytest.mark.parametrize("G", [32, 64])
+@pytest.mark.parametrize("G", [32, 64, 256])
 @pytest.mark.parametrize("idx", [0, 1])
 def test_group_sizes_full_workloads(idx, G, fmt):
     w = W.WORKLOADS[idx]
@@ -38,16 +41,16 @@ def test_group_sizes_full_workloads(idx, G, fmt):
     _check(x, gy, G, fmt, w.name)
 
 
-@pytest.mark.parametrize("G", [32, 64])
+@pytest.mark.parametrize("G", [32, 64, 256])
 @pytest.mark.parametrize("M,K", [(1, 128), (31, 384), (33, 128), (65, 256), (129, 128), (200, 384),
-                                 (257, 256), (1000, 128)])
+                                 (257, 256), (1000, 128), (513, 640), (300, 16)])
 def test_group_sizes_odd_and_tail_shapes(M, K, G):
     x, gy = W.make_inputs(W.small_workload(M, K, seed=M * 13 + K + G))
     _check(x, gy, G, (0, 0, 0), f"M={M} K={K}")
     _check(x, gy, G, (1, 1, 1), f"M={M} K={K}")
 
 
-@pytest.mark.parametrize("G", [32, 64])
+@pytest.mark.parametrize("G", [32, 64, 256])
 def test_group_sizes_outliers_zero_groups_and_tiny(G):
     x, gy = W.make_inputs(W.WORKLOADS[3])          # outliers, zero groups, a 32-token tail group
     _check(x, gy, G, (0, 0, 0), "outliers")
@@ -57,7 +60,7 @@ def test_group_sizes_outliers_zero_groups_and_tiny(G):
     _check(x, gy, G, (1, 1, 0), "tiny")
 
 
-@pytest.mark.parametrize("G", [32, 64])
+@pytest.mark.parametrize("G", [32, 64, 256])
 def test_group_sizes_over_the_whole_exponent_range(G):
     """gate = 32, grad_y = 1, up = a_i on token group i (of G tokens): the
     group amaxes sweep one bf16 value per exponent field, subnormals included."""
@@ -70,3 +73,11 @@ def test_group_sizes_over_the_whole_exponent_range(G):
     gy = np.full((M, K), 0x3F80, np.uint16)             # 1.0
     _check(x, gy, G, (0, 0, 0), "exponent sweep")
     _check(x, gy, G, (1, 1, 0), "exponent sweep")
+
+
+def test_group_256_on_the_outlier_workload_and_a_large_one():
+    """Groups of 256 on M=4000 K=2048 (outliers, zero groups, a 160-token tail
+    group) in full, and on M=8192 K=4096 in full, in the page's format."""
+    for idx in (3, 2):
+        x, gy = W.make_inputs(W.WORKLOADS[idx])
+        _check(x, gy, 256, (0, 0, 0), W.WORKLOADS[idx].name)

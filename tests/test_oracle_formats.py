@@ -214,7 +214,7 @@ def test_whole_op_fmt_ys_layouts_transpose(codes, scales):
         assert np.array_equal(u, v)
 
 
-@pytest.mark.parametrize("G", [128, 64, 32])
+@pytest.mark.parametrize("G", [256, 128, 64, 32])
 @pytest.mark.parametrize("codes,scales", FORMATS)
 def test_whole_op_fmt_groups_relate_to_stage1(codes, scales, G):
     # every group of all four outputs equals the exact restatement of the

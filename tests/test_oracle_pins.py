@@ -279,7 +279,7 @@ def _gate32_case(M, K):
 
 
 @pytest.mark.parametrize("M,K,G", [(200, 256, 128), (7, 128, 128), (129, 384, 128),
-                                   (200, 256, 64), (129, 128, 32)])
+                                   (200, 256, 64), (129, 128, 32), (300, 512, 256), (256, 256, 256)])
 def test_whole_op_gate32_closed_form(M, K, G):
     x, gy, a, w, e = _gate32_case(M, K)
     giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, G)

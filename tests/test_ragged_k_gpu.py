@@ -74,7 +74,8 @@ def _run(x_u16, gy_u16, G, fmt, with_y=False, int8_grad_y=None):
 
 
 @pytest.mark.parametrize("K", [16, 144, 208, 400, 1040])
-@pytest.mark.parametrize("G,fmt", [(128, (0, 0, 0)), (64, (1, 1, 1)), (32, (0, 1, 0)), (128, (1, 0, 1))])
+@pytest.mark.parametrize("G,fmt", [(128, (0, 0, 0)), (64, (1, 1, 1)), (32, (0, 1, 0)), (128, (1, 0, 1)),
+                                   (256, (0, 0, 0)), (256, (1, 1, 1))])
 def test_partial_channel_tile_matches_the_oracle(K, G, fmt):
     M = 300
     x, gy = W.make_inputs(W.small_workload(M, K, seed=K + G, zero_group_every=0))
@@ -92,16 +93,16 @@ def test_partial_channel_tile_large():
     U.compare_fmt(got, oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, 128, 0, 0, 0), 0, 0, 0, "K=1424")
 
 
-@pytest.mark.parametrize("K", [208, 1040])
-def test_partial_channel_tile_int8_grad_y_with_y(K):
+@pytest.mark.parametrize("K,G", [(208, 128), (1040, 128), (208, 256), (1040, 256), (400, 256)])
+def test_partial_channel_tile_int8_grad_y_with_y(K, G):
     M = 257
     w = W.small_workload(M, K, seed=3 * K, zero_group_every=5)
     x, _ = W.make_inputs(w)
     q, s = W.quantized_grad_y(w)
     assert s.shape == (M, (K + 127) // 128)
-    got = _run(x, None, 128, (0, 0, 0), with_y=True, int8_grad_y=(q, s))
-    U.compare_fmt(got[:4], oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, 128, 0, 0, 0), 0, 0, 0,
-                  f"int8 grad_y K={K}")
+    got = _run(x, None, G, (0, 0, 0), with_y=True, int8_grad_y=(q, s))
+    U.compare_fmt(got[:4], oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, G, 0, 0, 0), 0, 0, 0,
+                  f"int8 grad_y K={K} G={G}", G)
     U.compare_bf16(got[4], oracle.swiglu_bwd_bf16_dy(x, oracle.dequant_grad_y(q, s))[0], "y", f"K={K}")
 
 
