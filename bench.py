@@ -71,6 +71,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["sdq", "reference"], default="sdq")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--group-size", type=int, default=128, choices=[32, 64, 128, 256],
+                    help="the page's group_size argument for the timed calls (default 128)")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the per_workload list (every workload timed after the headline)")
     ap.add_argument("--per-workload-ms", type=float, default=50.0,
@@ -359,14 +361,14 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
         xs = x0 if s == 0 else x0.clone()
         gs = g0 if s == 0 else g0.clone()
         gss = gs0 if (s == 0 or gs0 is None) else gs0.clone()
-        sets.append((xs, gs, gss, sdq.allocate_outputs(M, K, device, codes=codes, scales=scales,
-                                                       y_scale_layout=layout),
+        sets.append((xs, gs, gss, sdq.allocate_outputs(M, K, device, group_size=w.group_size, codes=codes,
+                                                       scales=scales, y_scale_layout=layout),
                      torch.empty(M, K, dtype=torch.bfloat16, device=device) if with_y else None))
     stream = torch.cuda.current_stream(device)
 
     def call(k):
         xs, gs, gss, outs, ys = sets[k % nsets]
-        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, codes=codes, scales=scales,
+        sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, w.group_size, codes=codes, scales=scales,
                                         y_scale_layout=layout, y=ys, grad_y_s=gss)
 
     for k in range(warmup):
@@ -442,6 +444,9 @@ def run_sdq(args):
     parallel.init_from_env("nccl", timeout_s=120.0, device=device)
 
     w = pick_workload(args.workload)
+    if args.group_size != w.group_size:   # same inputs, another group size
+        w = W.Workload(w.name, w.M, w.K, w.sigma_x, w.sigma_grad_y, w.seed, args.group_size,
+                       w.outlier_frac, w.outlier_mult, w.zero_group_every)
     # Each rank its own replica (seed offset by rank): weak scaling, no exchange.
     wr = W.Workload(w.name, w.M, w.K, w.sigma_x, w.sigma_grad_y, w.seed + 1000 * rank,
                     w.group_size, w.outlier_frac, w.outlier_mult, w.zero_group_every)

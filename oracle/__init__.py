@@ -143,19 +143,20 @@ def swiglu_bwd_bf16(x: np.ndarray, grad_y: np.ndarray):
 
 
 def silu_dot_fwd_bwd_quant_fuse(x: np.ndarray, grad_y: np.ndarray, group_size: int = 128):
-    """The whole op on uint16 (bf16 bit) arrays.
+    """The whole op on uint16 (bf16 bit) arrays, in the page's format.
 
-    Returns ``(grad_input_q [M,2K] int8, grad_input_s [M,2K/G] f32,
-    y_q_t [K,M] int8, y_s_t [K,ceil(M/G)] f32)``.
+    Returns ``(grad_input_q [M,2K] int8, grad_input_s [M,2 ceil(K/G)] f32,
+    y_q_t [K,M] int8, y_s_t [K,ceil(M/G)] f32)``; when G does not divide K
+    the last channel group of each half of [d_gate | d_up] is shorter.
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     gy = np.ascontiguousarray(grad_y, dtype=np.uint16)
     M, K = gy.shape
     assert x.shape == (M, 2 * K), (x.shape, gy.shape)
     G = int(group_size)
-    if G < 1 or K % G:
-        raise ValueError(f"K={K} is not a multiple of group_size={G}")
-    Kg, Mg = K // G, (M + G - 1) // G
+    if G < 1:
+        raise ValueError(f"group_size={G} must be positive")
+    Kg, Mg = (K + G - 1) // G, (M + G - 1) // G
     giq = np.zeros((M, 2 * K), np.int8)
     gis = np.zeros((M, 2 * Kg), np.float32)
     yqt = np.zeros((K, M), np.int8)

@@ -22,8 +22,9 @@
 // once, to nearest even; scale = amax/127 in fp32; q = round-half-even of the
 // fp32 quotient v/scale, clamped to [-127, 127]; an all-zero group gets
 // scale 1 and q 0; a tail token group (M % G != 0) is quantized over the
-// tokens it holds; grad_input_s is [M, 2K/G] (d_gate groups first) and
-// y_s_t is [K, ceil(M/G)].
+// tokens it holds, and likewise a channel group cut short by the end of its
+// half of [d_gate | d_up] when G does not divide K; grad_input_s is
+// [M, 2 ceil(K/G)] (d_gate groups first) and y_s_t is [K, ceil(M/G)].
 //
 // How each function is pinned (tests/test_oracle_pins.py):
 //   oracle_bf16_rne        brute force over the neighbouring bf16 values with
@@ -34,9 +35,10 @@
 //   oracle_silu_grad       central finite difference of oracle_silu.
 //   oracle_swiglu_bwd_fp64 torch float64 autograd of sum(grad_y*silu(g)*u);
 //                          finite differences of y in g and u.
-//   oracle_quant_group     exact-rational check that scale is amax/127
-//                          rounded once, nearest-integer brute force, exact
-//                          ties to even, symmetry and monotonicity.
+//   oracle_quant_group     (the page's format of oracle_quant_group_fmt, the
+//                          one quantizer) exact-rational check that scale is
+//                          amax/127 rounded once, nearest-integer brute
+//                          force, exact ties to even, symmetry, monotonicity.
 //   whole op               closed-form hand-derived cases (gate = 0, gate
 //                          large), layout/transposition patterns, tail and
 //                          zero groups, and a hand-derived golden fixture.
@@ -149,33 +151,6 @@ void oracle_swiglu_bwd_fp64(double g, double u, double dy, double* y,
   *d_up = dy * silu;
 }
 
-// Quantize one group of n bf16 values (element i at v[i*stride]) to int8:
-// amax = max |v|; all-zero -> scale 1, q 0; else scale = amax/127 (fp32
-// division) and q = clamp(round-half-even(v/scale), -127, 127) with the
-// quotient taken in fp32.  Writes q[i*qstride] and *scale.
-void oracle_quant_group(const uint16_t* v, int64_t n, int64_t stride,
-                        int8_t* q, int64_t qstride, float* scale) {
-  float amax = 0.0f;
-  for (int64_t i = 0; i < n; ++i) {
-    const float a = std::fabs(bf16_to_float(v[i * stride]));
-    if (a > amax) amax = a;
-  }
-  if (amax == 0.0f) {
-    *scale = 1.0f;
-    for (int64_t i = 0; i < n; ++i) q[i * qstride] = 0;
-    return;
-  }
-  const float s = amax / 127.0f;
-  for (int64_t i = 0; i < n; ++i) {
-    const float t = bf16_to_float(v[i * stride]) / s;
-    float r = std::nearbyint(t);
-    if (r > 127.0f) r = 127.0f;
-    if (r < -127.0f) r = -127.0f;
-    q[i * qstride] = static_cast<int8_t>(r);
-  }
-  *scale = s;
-}
-
 // First stage on grad_y given as fp64 values dy [M, K]: the bf16 values y,
 // d_gate, d_up ([M, K] each, bf16 bits) from x = [gate | up] ([M, 2K]).
 void oracle_swiglu_bwd_bf16_dy(const uint16_t* x, const double* dy, int64_t M, int64_t K,
@@ -200,43 +175,6 @@ void oracle_swiglu_bwd_bf16(const uint16_t* x, const uint16_t* grad_y,
   std::vector<double> dy(M * K);
   for (int64_t i = 0; i < M * K; ++i) dy[i] = bf16_to_float(grad_y[i]);
   oracle_swiglu_bwd_bf16_dy(x, dy.data(), M, K, y, d_gate, d_up);
-}
-
-// The whole op.  Returns 0, or -1 for arguments the definition does not cover
-// (group_size < 1, K not a multiple of group_size, negative sizes).
-//   grad_input_q [M, 2K] int8     grad_input_s [M, 2K/G] fp32
-//   y_q_t        [K, M]  int8     y_s_t        [K, ceil(M/G)] fp32
-int oracle_silu_dot_fwd_bwd_quant_fuse(const uint16_t* x, const uint16_t* grad_y,
-                                       int8_t* grad_input_q, float* grad_input_s,
-                                       int8_t* y_q_t, float* y_s_t, int64_t M,
-                                       int64_t K, int64_t group_size) {
-  const int64_t G = group_size;
-  if (G < 1 || M < 0 || K < 0 || K % G != 0) return -1;
-  if (M == 0 || K == 0) return 0;
-  const int64_t Kg = K / G;
-  const int64_t Mg = (M + G - 1) / G;
-  std::vector<uint16_t> y(M * K), dg(M * K), du(M * K);
-  oracle_swiglu_bwd_bf16(x, grad_y, M, K, y.data(), dg.data(), du.data());
-
-  // Row-wise: token m, group j of the 2K channels of [d_gate | d_up].
-  for (int64_t m = 0; m < M; ++m) {
-    for (int64_t j = 0; j < 2 * Kg; ++j) {
-      const uint16_t* src = (j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G];
-      oracle_quant_group(src, G, 1, &grad_input_q[m * 2 * K + j * G], 1,
-                         &grad_input_s[m * 2 * Kg + j]);
-    }
-  }
-  // Column-wise on y: channel k, token group i (the tail group holds M - i*G tokens);
-  // stored transposed, y_q_t[k, t] for token t.
-  for (int64_t k = 0; k < K; ++k) {
-    for (int64_t i = 0; i < Mg; ++i) {
-      const int64_t t0 = i * G;
-      const int64_t n = (M - t0 < G) ? (M - t0) : G;
-      oracle_quant_group(&y[t0 * K + k], n, K, &y_q_t[k * M + t0], 1,
-                         &y_s_t[k * Mg + i]);
-    }
-  }
-  return 0;
 }
 
 // ---- output formats ---------------------------------------------------------
@@ -322,6 +260,15 @@ void oracle_quant_group_fmt(const uint16_t* v, int64_t n, int64_t stride, uint8_
   }
 }
 
+// The page's format of oracle_quant_group_fmt: INT8 codes (q as int8),
+// fp32 scale.  amax = max |v|; all-zero -> scale 1, q 0; else scale =
+// amax/127 (fp32 division) and q = clamp(round-half-even(v/scale), -127, 127)
+// with the quotient taken in fp32.  Writes q[i*qstride] and *scale.
+void oracle_quant_group(const uint16_t* v, int64_t n, int64_t stride,
+                        int8_t* q, int64_t qstride, float* scale) {
+  oracle_quant_group_fmt(v, n, stride, reinterpret_cast<uint8_t*>(q), qstride, scale, 0, 0);
+}
+
 // The whole op in a chosen format.  codes / scales as in
 // oracle_quant_group_fmt; ys_layout: 0 y_s_t [K, Mg], 1 [Mg, K].  Code
 // arrays are bytes; scale arrays are fp32 or one byte per scale.
@@ -344,6 +291,21 @@ int oracle_silu_dot_fwd_bwd_quant_fuse_fmt(const uint16_t* x, const uint16_t* gr
   quantize_outputs_fmt(y.data(), dg.data(), du.data(), grad_input_q, grad_input_s, y_q_t, y_s_t,
                        M, K, G, codes, scales, ys_layout);
   return 0;
+}
+
+// The whole op in the page's format (INT8 codes, fp32 scales, y_s_t
+// [K, ceil(M/G)]): the format op above with codes 0, scales 0, layout 0.
+// Returns 0, or -1 for arguments the definition does not cover
+// (group_size < 1, negative sizes).
+//   grad_input_q [M, 2K] int8     grad_input_s [M, 2 ceil(K/G)] fp32
+//   y_q_t        [K, M]  int8     y_s_t        [K, ceil(M/G)] fp32
+int oracle_silu_dot_fwd_bwd_quant_fuse(const uint16_t* x, const uint16_t* grad_y,
+                                       int8_t* grad_input_q, float* grad_input_s,
+                                       int8_t* y_q_t, float* y_s_t, int64_t M,
+                                       int64_t K, int64_t group_size) {
+  return oracle_silu_dot_fwd_bwd_quant_fuse_fmt(x, grad_y, reinterpret_cast<uint8_t*>(grad_input_q),
+                                                grad_input_s, reinterpret_cast<uint8_t*>(y_q_t), y_s_t,
+                                                M, K, group_size, 0, 0, 0);
 }
 
 // ---- grad_y handed over already quantized (the chained backward) -------------

@@ -20,16 +20,18 @@ MUTATIONS = [
     ("*d_gate = dy * u * oracle_silu_grad(g);", "*d_gate = dy * oracle_silu_grad(g);", "test_swiglu_bwd_fp64_finite_differences"),
     ("*d_up = dy * silu;", "*d_up = dy * u;", "test_swiglu_bwd_fp64_matches_torch_autograd"),
     ("x[m * 2 * K + k]);", "x[m * 2 * K + K + k]);", "test_whole_op_gate32_closed_form"),
-    ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;", "test_quant_scale_is_amax_over_127_rounded_once"),
+    ("const float qmax = codes ? 448.0f : 127.0f;", "const float qmax = codes ? 448.0f : 128.0f;",
+     "test_quant_scale_is_amax_over_127_rounded_once"),
     ("float r = std::nearbyint(t);", "float r = std::round(t);", "test_quant_ties_to_even_and_symmetry"),
     ("(j < Kg) ? &dg[m * K + j * G] : &du[m * K + (j - Kg) * G]",
      "(j < Kg) ? &du[m * K + j * G] : &dg[m * K + (j - Kg) * G]", "test_whole_op_gate32_closed_form"),
     ("&y_q_t[k * M + t0], 1,", "&y_q_t[t0 * K + k], K,", "test_whole_op_gate32_closed_form"),
-    ("&y_s_t[k * Mg + i]", "&y_s_t[i * K + k]", "test_whole_op_gate32_closed_form"),
-    ("&grad_input_s[m * 2 * Kg + j]", "&grad_input_s[j * M + m]", "test_whole_op_groups_relate_to_stage1"),
+    ("const int64_t si = ys_layout ? (i * K + k) : (k * Mg + i);",
+     "const int64_t si = ys_layout ? (i * K + k) : (i * K + k);", "test_whole_op_gate32_closed_form"),
+    ("gis + (m * 2 * Kg + j) * sb", "gis + (j * M + m) * sb", "test_whole_op_groups_relate_to_stage1"),
     ("const double r = std::nearbyint(a / ulp) * ulp;", "const double r = std::trunc(a / ulp) * ulp;",
      "test_bf16_rne_bruteforce_exact_rationals"),
-    ("*scale = 1.0f;", "*scale = 0.0f;", "test_quant_zero_and_constant_groups"),
+    ("    s = 1.0;\n", "    s = 2.0;\n", "test_quant_zero_and_constant_groups"),
     ("if (e < -126) e = -126;", "", "test_bf16_rne_against_torch_float32_conversion"),
     ("return 1.0 / (1.0 + std::exp(-g));", "return 1.0 / (1.0 + std::exp(-(float)g));",
      "test_sigmoid_matches_library_expit"),
@@ -72,7 +74,7 @@ MUTATIONS = [
     # the whole op against its brute-force restatement (test_oracle_bruteforce.py)
     ("*d_up = dy * silu;", "*d_up = dy * silu * u;", "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
     ("x[m * 2 * K + k]);", "x[m * 2 * K + K + k]);", "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
-    ("const float s = amax / 127.0f;", "const float s = amax / 127.5f;",
+    ("const float qmax = codes ? 448.0f : 127.0f;", "const float qmax = codes ? 448.0f : 127.5f;",
      "test_whole_oracle_equals_bruteforce_on_4x128", "brute"),
     # groups of G channels when G does not divide K (pins in test_oracle_formats.py)
     ("const int64_t n = (K - c0 < G) ? K - c0 : G;", "const int64_t n = G < K ? G : K;",

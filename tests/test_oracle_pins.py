@@ -384,11 +384,19 @@ def test_whole_op_groups_relate_to_stage1():
         assert np.all(np.abs(deq - blk.T) <= yst[:, i:i + 1] * (0.5 + 2 ** -15))
 
 
-def test_rejects_k_not_multiple_of_group():
+def test_page_format_is_the_format_op_at_int8_fp32():
+    """The page-format entry is the format op with INT8 codes, fp32 scales and
+    y_s_t [K, Mg] (one quantizer), also where G does not divide K (a shorter
+    last channel group in each half); a group size below 1 is rejected."""
+    for M, K, G, seed in [(40, 256, 128, 1), (37, 100, 128, 2), (20, 100, 50, 3), (9, 208, 64, 4)]:
+        x, gy = W.make_inputs(W.small_workload(M, K, seed=seed))
+        a = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, group_size=G)
+        b = oracle.silu_dot_fwd_bwd_quant_fuse_fmt(x, gy, G, 0, 0, 0)
+        Kg = (K + G - 1) // G
+        assert a[1].shape == (M, 2 * Kg) and a[3].shape == (K, (M + G - 1) // G)
+        assert np.array_equal(a[0].view(np.uint8), b[0]) and np.array_equal(a[2].view(np.uint8), b[2])
+        assert np.array_equal(a[1], b[1]) and np.array_equal(a[3], b[3])
     x = np.zeros((4, 2 * 100), np.uint16)
     gy = np.zeros((4, 100), np.uint16)
     with pytest.raises(ValueError):
-        oracle.silu_dot_fwd_bwd_quant_fuse(x, gy)
-    # a different group size is a different (valid) definition
-    giq, gis, yqt, yst = oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, group_size=50)
-    assert gis.shape == (4, 4) and yst.shape == (100, 1)
+        oracle.silu_dot_fwd_bwd_quant_fuse(x, gy, group_size=0)

@@ -37,6 +37,8 @@ _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 _CHUNK = 1 << 22
 
+ZERO_GROUP_WIDTH = 128   # channels zeroed (in gate and up) per zero-group row, whatever the group size
+
 STREAM_X = 0
 STREAM_GRAD_Y = 1
 STREAM_OUTLIER = 2
@@ -160,7 +162,8 @@ class Workload:
         (m, k)), write grad_input_q (2 B) and y_q_t (1 B) codes, plus the
         scales (fp32: 4 B each; E8M0: 1 B)."""
         mk = self.M * self.K
-        return 6 * mk + 3 * mk + scale_bytes * (self.M * 2 * self.Kg + self.K * self.Mg)
+        kgs = (self.K + self.group_size - 1) // self.group_size   # row groups per half (last may be short)
+        return 6 * mk + 3 * mk + scale_bytes * (self.M * 2 * kgs + self.K * self.Mg)
 
     def describe(self) -> Dict[str, object]:
         return {"workload": self.name, "M": self.M, "K": self.K,
@@ -200,11 +203,12 @@ def make_inputs(w: Workload) -> Tuple[np.ndarray, np.ndarray]:
             if hit.size:
                 v = bf16_bits_to_f32(flat[hit]) * np.float32(w.outlier_mult)
                 flat[hit] = f32_to_bf16_bits(v)
-    if w.zero_group_every > 0 and w.Kg > 0:
+    nz = K // ZERO_GROUP_WIDTH
+    if w.zero_group_every > 0 and nz > 0:
         key = stream_key(w.seed, STREAM_ZERO_GROUP)
         rows = np.arange(0, M, w.zero_group_every)
-        groups = (draws(key, 0, rows.size) % np.uint64(w.Kg)).astype(np.int64)
-        G = w.group_size
+        groups = (draws(key, 0, rows.size) % np.uint64(nz)).astype(np.int64)
+        G = ZERO_GROUP_WIDTH
         for r, j in zip(rows.tolist(), groups.tolist()):
             x[r, j * G:(j + 1) * G] = 0          # gate
             x[r, K + j * G:K + (j + 1) * G] = 0  # up
@@ -213,11 +217,12 @@ def make_inputs(w: Workload) -> Tuple[np.ndarray, np.ndarray]:
 
 def zero_group_positions(w: Workload) -> List[Tuple[int, int]]:
     """(row, group) pairs zeroed by ``make_inputs`` (for tests of the all-zero case)."""
-    if w.zero_group_every <= 0 or w.Kg == 0:
+    nz = w.K // ZERO_GROUP_WIDTH
+    if w.zero_group_every <= 0 or nz == 0:
         return []
     key = stream_key(w.seed, STREAM_ZERO_GROUP)
     rows = np.arange(0, w.M, w.zero_group_every)
-    groups = (draws(key, 0, rows.size) % np.uint64(w.Kg)).astype(np.int64)
+    groups = (draws(key, 0, rows.size) % np.uint64(nz)).astype(np.int64)
     return list(zip(rows.tolist(), groups.tolist()))
 
 
