@@ -16,12 +16,16 @@
 
 namespace {
 
-// Pipeline depth of the kernel's shared-memory ring (48 KB per stage;
-// compile-time overridable for tuning sweeps).
+// Pipeline depth of the kernels' shared-memory rings (48 KB per stage;
+// compile-time overridable for tuning sweeps): three for the 128 x 128-tile
+// kernel (its two warp halves work on different slots, and a third slot
+// keeps a load in flight for each), two for the 256-group kernel (its 128 KB
+// y buffer leaves no room for a third).
 #ifndef SDQ_STAGES
-#define SDQ_STAGES 2
+#define SDQ_STAGES 3
 #endif
 constexpr int kStages = SDQ_STAGES;
+constexpr int kStages256 = 2;
 
 constexpr int kMaxDevices = 64;
 
@@ -51,14 +55,14 @@ constexpr KernelFn kernel_of(int f) {
 template <bool kY, bool kQ>
 constexpr KernelFn kernel256_of(int f) {
   switch (f) {
-    case 0: return sdq::fuse256_kernel<kStages, false, false, false, kY, kQ>;
-    case 1: return sdq::fuse256_kernel<kStages, true, false, false, kY, kQ>;
-    case 2: return sdq::fuse256_kernel<kStages, false, true, false, kY, kQ>;
-    case 3: return sdq::fuse256_kernel<kStages, true, true, false, kY, kQ>;
-    case 4: return sdq::fuse256_kernel<kStages, false, false, true, kY, kQ>;
-    case 5: return sdq::fuse256_kernel<kStages, true, false, true, kY, kQ>;
-    case 6: return sdq::fuse256_kernel<kStages, false, true, true, kY, kQ>;
-    default: return sdq::fuse256_kernel<kStages, true, true, true, kY, kQ>;
+    case 0: return sdq::fuse256_kernel<kStages256, false, false, false, kY, kQ>;
+    case 1: return sdq::fuse256_kernel<kStages256, true, false, false, kY, kQ>;
+    case 2: return sdq::fuse256_kernel<kStages256, false, true, false, kY, kQ>;
+    case 3: return sdq::fuse256_kernel<kStages256, true, true, false, kY, kQ>;
+    case 4: return sdq::fuse256_kernel<kStages256, false, false, true, kY, kQ>;
+    case 5: return sdq::fuse256_kernel<kStages256, true, false, true, kY, kQ>;
+    case 6: return sdq::fuse256_kernel<kStages256, false, true, true, kY, kQ>;
+    default: return sdq::fuse256_kernel<kStages256, true, true, true, kY, kQ>;
   }
 }
 
@@ -94,7 +98,7 @@ KernelFn kernel_for(int32_t group_size, uint32_t format, bool y, bool qdy) {
 
 // Dynamic shared memory of the kernel for a group size.
 size_t smem_for(int32_t group_size) {
-  return group_size == 256 ? sdq::smem_bytes256<kStages>() : sdq::smem_bytes<kStages>();
+  return group_size == 256 ? sdq::smem_bytes256<kStages256>() : sdq::smem_bytes<kStages>();
 }
 
 bool group_size_supported(int32_t g) { return g == 32 || g == 64 || g == SDQ_GROUP_SIZE || g == 256; }
@@ -160,7 +164,7 @@ int current_device(DeviceState** out) {
     d.init_err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     for (int n = 0; n < kKernels; ++n) {
       const auto kernel = kernel_at(n);
-      const size_t smem = is_group256(n) ? sdq::smem_bytes256<kStages>() : sdq::smem_bytes<kStages>();
+      const size_t smem = is_group256(n) ? sdq::smem_bytes256<kStages256>() : sdq::smem_bytes<kStages>();
       if (d.init_err == cudaSuccess)
         d.init_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(smem));

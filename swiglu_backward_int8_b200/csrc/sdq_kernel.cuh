@@ -30,13 +30,18 @@
 //     warp, so every warp computes and may use 128 registers.
 //     Rows past M are zero-filled by the TMA unit, and zeros never change an
 //     amax, so a tail token group is quantized over exactly the tokens it holds.
-//   * row pass: a lane owns 16 channels of one token row per stage (8 lanes per
-//     row, 4 rows per warp): fp32 math in packed f32x2 instructions, bf16
-//     rounding, the row amax of d_gate and d_up by a 3-step shuffle reduction
-//     on packed bf16 pairs, each lane computing its row's two scales itself
-//     (no shuffles), quantization by multiplication with the inverse scale,
-//     coalesced stores; the bf16 y values go to a shared [token][channel]
-//     tile (double-buffered across tiles).
+//   * row pass: warps 0-7 take the first stage of every tile and warps 8-15
+//     the second, so the two halves of the CTA work on different slots and a
+//     slot waits for 8 warps, not 16.  A lane owns 32 channels of one token
+//     row (4 lanes per row, 8 rows per warp): fp32 math in packed f32x2
+//     instructions, bf16 rounding, the row amax of d_gate and d_up over its
+//     chunks and then over the row's 4 lanes (2 shuffle steps on packed bf16
+//     pairs), each lane computing its row's scales itself, quantization by
+//     multiplication with the inverse scale, 8-byte stores per 8 channels; the
+//     bf16 y values go to a shared [token][channel] tile (double-buffered
+//     across tiles).  Per-row work (reductions, scales, the stage's wait and
+//     release) is spread over 32 elements a lane, half the cost per element
+//     of 16-channel lanes.
 //   * column pass, one tile late (after the row pass of the next tile, so no
 //     warp waits for the others at a tile boundary; two mbarriers per y buffer
 //     say "all rows written" and "all columns read"): a thread owns 2 channels
@@ -44,9 +49,10 @@
 //     share its channels, computes the two column scales, quantizes its 32 y
 //     values and stores two 16-byte pieces of y_q_t rows; each group of 8
 //     threads writes one 128-byte line.
-//   * shared-memory layouts are chosen for conflict-free access: a lane of the
-//     upper half of an 8-lane row group takes its two 16-byte chunks in the
-//     opposite order, and the y tile's chunks are XOR-swizzled by token.
+//   * shared-memory layouts are chosen for conflict-free access: a lane of an
+//     odd row takes its chunks in the order (4k + q) ^ 4, so each 8-lane
+//     quarter of a warp reads 8 distinct bank groups, and the y tile's chunks
+//     are XOR-swizzled by token.
 //
 // Every wait on an mbarrier is bounded (Params::wait_limit_ns).  A wait that
 // runs out sets the device status word and a shared abort flag that every
@@ -69,7 +75,6 @@ constexpr int kQBoxBytes = kStageRows * kG;         // one INT8 grad_y box: 8 KB
 constexpr int kYBytes = kG * kG * 2;                // bf16 y tile: 32 KB
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRowsPerWarp = kStageRows / kWarps;   // 4 (8 lanes per row)
 #ifndef SDQ_YBUF
 #define SDQ_YBUF 2
 #endif
@@ -454,25 +459,77 @@ __device__ __forceinline__ void column_pass(const uint8_t* yt, const float2* tab
   }
 }
 
+// Eight codes of one 16-byte chunk (4 bf16 pairs) with one inverse scale;
+// `scale` as in quant16.
+template <bool kE4M3, bool kTiny>
+__device__ __forceinline__ uint2 quant8(const uint32_t* v, float inv, float scale) {
+  const float2 iv = make_float2(inv, inv);
+  const float2 pre = make_float2(kTinyPre, kTinyPre);
+  const float2 sc = make_float2(scale, scale);
+  return make_uint2(pack_codes<kE4M3>(quant2<kE4M3, kTiny>(v[0], iv, pre, sc), quant2<kE4M3, kTiny>(v[1], iv, pre, sc)),
+                    pack_codes<kE4M3>(quant2<kE4M3, kTiny>(v[2], iv, pre, sc), quant2<kE4M3, kTiny>(v[3], iv, pre, sc)));
+}
+
+// Tile sequence of this CTA (tiles blockIdx.x, blockIdx.x + gridDim.x, ...)
+// in the banded order of tile_ij, stepped without a division per tile: the
+// position within the current band advances by gridDim.x and wraps into
+// the next band.
+struct TileWalk {
+  int bsz;    // tiles per band: kBand * Kg
+  int band;
+  int r;      // position inside the band
+  __device__ __forceinline__ void start(int t, int Kg) {
+    bsz = SDQ_TILE_BAND * Kg;
+    band = t / bsz;
+    r = t - band * bsz;
+  }
+  __device__ __forceinline__ void next() {
+    r += gridDim.x;
+    while (r >= bsz) {
+      r -= bsz;
+      ++band;
+    }
+  }
+  __device__ __forceinline__ void ij(int Mg, int& i, int& j) const {
+    constexpr int kBand = SDQ_TILE_BAND;
+    const int rows = min(kBand, Mg - band * kBand);
+    if (rows == kBand) {
+      i = band * kBand + (r & (kBand - 1));
+      j = r / kBand;
+    } else {
+      i = band * kBand + r % rows;
+      j = r / rows;
+    }
+  }
+};
+
 template <int STAGES, int kGS, bool kE4M3, bool kE8M0, bool kYsMgK, bool kY, bool kQdy>
 __global__ void __launch_bounds__(kThreads, 1)
     fuse_kernel(const __grid_constant__ CUtensorMap map_gate, const __grid_constant__ CUtensorMap map_up,
                 const __grid_constant__ CUtensorMap map_gy,
                 const Params p) {
   constexpr unsigned kFull = 0xffffffffu;
+  constexpr int kNG = kG / kGS;     // row groups per tensor in a tile row: 1, 2, 4
+  constexpr int kSPG = 4 / kNG;     // a lane's chunks per group: 4, 2, 1
   extern __shared__ uint8_t smem_raw[];
   auto& s = *reinterpret_cast<Smem<STAGES>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  // row pass: lane = 8 * rr + cq owns 16-byte chunks ca, cb (8 channels each)
-  // of row srow; the upper half of the row group takes them in swapped order
-  const int rr = lane >> 3;
-  const int cq = lane & 7;
-  const int ca = 2 * cq + (cq >> 2);
-  const int cb = 2 * cq + 1 - (cq >> 2);
-  const int srow = warp * kRowsPerWarp + rr;
+  // row pass: warps 0-7 take stage 0 of every tile, warps 8-15 stage 1; lane
+  // (rr, q) of warp wi owns row 8 wi + rr of the stage and its 16-byte chunks
+  // ch[k] = (4k + q) ^ 4 (rr & 1), k = 0..3 (8 channels each): an 8-lane
+  // quarter of the warp then reads 8 distinct bank groups
+  const int grp = warp >> 3;
+  const int rr = lane >> 2;
+  const int q = lane & 3;
+  const int par = rr & 1;
+  const int srow = (warp & 7) * 8 + rr;
+  const int r = grp * kStageRows + srow;   // this lane's row within the tile
+  int ch[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ch[k] = (4 * k + q) ^ (4 * par);
   // column pass: thread = 8 * cp + kc owns channels 2cp, 2cp+1 and tokens 16kc..16kc+15
   const int cp = tid >> 3;
   const int kc = tid & 7;
@@ -507,7 +564,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   const int K = p.K;
-  const int Kg = p.Kg;
   const int64_t M = p.M;
   const float2* tab = s.scale_tab;
   volatile int* abort_flag = &s.abort;
@@ -522,153 +578,165 @@ __global__ void __launch_bounds__(kThreads, 1)
   // each other in a cycle.
   int pi = 0, pj = 0, pvalid = 0;   // the tile whose column pass is pending
   int64_t prow0 = 0;
+  TileWalk walk;
+  walk.start(blockIdx.x, p.Kg);
 
   for (int k = 0; k < my_tiles && ok; ++k) {
-    const int t = blockIdx.x + k * gridDim.x;
+    if (k > 0) walk.next();
     int i, j;
-    tile_ij(t, p.Mg, Kg, i, j);
+    walk.ij(p.Mg, i, j);
     const int64_t row0 = int64_t(i) * kG;
     const int valid = static_cast<int>(M - row0 < kG ? M - row0 : int64_t(kG));
-    const int cvalid = min(kG, K - j * kG);   // channels of this tile (K % 128 != 0: fewer in the last)
+    const int cvalid = min(kG, K - j * kG);   // channels of this tile (fewer in a partial last one)
     const int yb = k % kYBuf;   // y buffer of this tile; tile t completes phase t / kYBuf of its barriers
-    uint8_t* yt = s.ytile[yb];
-    // this tile's pieces of the row outputs (64-bit once per tile, 32-bit offsets per row)
-    int8_t* giq_t = p.giq + row0 * p.ld_giq + j * kG;
-    // scale index of (row0, the tile's first d_gate group)
-    const int64_t gis_t = row0 * p.ld_gis + j * (kG / kGS);
+    const uint32_t n = static_cast<uint32_t>(k) * kStagesPerTile + grp;   // this warp's load
+    const uint32_t slot = n % STAGES;
+    float dsc = 0.0f;   // INT8 grad_y: the scale of this lane's row in tile column j
+    if constexpr (kQdy) {
+      if (r < valid) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + j);
+    }
+    ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
+    if (!ok) break;
 
-    // ================= row pass over the tile's two stages
+    // ---- stage -> registers, then release the slot (the last of the 8 warps refills it)
+    uint4 gv[4], uv[4], dv[4];
+    float2 dq[16];   // INT8 grad_y, dequantized
+    {
+      const uint8_t* src = s.ring[slot] + srow * (kG * 2);
 #pragma unroll
-    for (int sub = 0; sub < kStagesPerTile; ++sub) {
-      const uint32_t n = static_cast<uint32_t>(k) * kStagesPerTile + sub;
-      const uint32_t slot = n % STAGES;
-      float dsc = 0.0f;   // INT8 grad_y: the scale of this lane's row in tile column j
-      if constexpr (kQdy) {
-        const int r = sub * kStageRows + srow;
-        if (r < valid) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + j);
-      }
-      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
-      if (!ok) break;
-
-      // ---- stage -> registers, then release the slot (the last warp refills it)
-      uint32_t gw[8], uw[8], dw[8];
-      float2 dq[8];   // INT8 grad_y, dequantized
-      {
-        const uint8_t* src = s.ring[slot] + srow * (kG * 2);
-        const uint4 g0 = *reinterpret_cast<const uint4*>(src + ca * 16);
-        const uint4 g1 = *reinterpret_cast<const uint4*>(src + cb * 16);
-        const uint4 u0 = *reinterpret_cast<const uint4*>(src + kBoxBytes + ca * 16);
-        const uint4 u1 = *reinterpret_cast<const uint4*>(src + kBoxBytes + cb * 16);
-        gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w;
-        gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
-        uw[0] = u0.x; uw[1] = u0.y; uw[2] = u0.z; uw[3] = u0.w;
-        uw[4] = u1.x; uw[5] = u1.y; uw[6] = u1.z; uw[7] = u1.w;
-        if constexpr (kQdy) {   // codes of row srow: 128 bytes, 8 per chunk
+      for (int c = 0; c < 4; ++c) {
+        gv[c] = *reinterpret_cast<const uint4*>(src + ch[c] * 16);
+        uv[c] = *reinterpret_cast<const uint4*>(src + kBoxBytes + ch[c] * 16);
+        if constexpr (kQdy) {
           const uint8_t* qsrc = s.ring[slot] + 2 * kBoxBytes + srow * kG;
-          dequant8(*reinterpret_cast<const uint2*>(qsrc + ca * 8), dsc, dq);
-          dequant8(*reinterpret_cast<const uint2*>(qsrc + cb * 8), dsc, dq + 4);
+          dequant8(*reinterpret_cast<const uint2*>(qsrc + ch[c] * 8), dsc, dq + 4 * c);
         } else {
-          const uint4 d0 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + ca * 16);
-          const uint4 d1 = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + cb * 16);
-          dw[0] = d0.x; dw[1] = d0.y; dw[2] = d0.z; dw[3] = d0.w;
-          dw[4] = d1.x; dw[5] = d1.y; dw[6] = d1.z; dw[7] = d1.w;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        if (atomicAdd(&s.released[slot], 1) == kWarps - 1) {
-          __threadfence_block();
-          s.released[slot] = 0;
-          const uint32_t nn = n + STAGES;
-          if (nn < total) {
-            atomicMax(&s.issued, static_cast<int>(nn + 1));
-            issue_load<STAGES, kQdy>(s, &map_gate, &map_up, &map_gy, p, nn, pol);
-          }
-        }
-      }
-
-      // ---- math, bf16 rounding
-      uint32_t yv[8], dgp[8], dup[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if constexpr (kQdy) swiglu_bwd2f(gw[c], uw[c], dq[c], yv[c], dgp[c], dup[c]);
-        else swiglu_bwd2(gw[c], uw[c], dw[c], yv[c], dgp[c], dup[c]);
-      }
-
-      // ---- y to the shared tile (chunks swizzled by token); the buffer was
-      // last read by the column pass of tile k - kYBuf
-      if (sub == 0 && k >= kYBuf) {
-        ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_free[yb]), (k / kYBuf - 1) & 1, lim,
-                                             abort_flag));
-        if (!ok) break;
-      }
-      {
-        const int tok = sub * kStageRows + srow;
-        const int key = (tok >> 4) & 7;
-        uint8_t* yrow = yt + tok * (kG * 2);
-        *reinterpret_cast<uint4*>(yrow + (ca ^ key) * 16) = make_uint4(yv[0], yv[1], yv[2], yv[3]);
-        *reinterpret_cast<uint4*>(yrow + (cb ^ key) * 16) = make_uint4(yv[4], yv[5], yv[6], yv[7]);
-      }
-      if constexpr (kY) {   // y itself, bf16 (optional output): 16 bytes per chunk
-        const int yr = sub * kStageRows + srow;
-        if (yr < valid) {
-          int8_t* yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + yr) * p.ld_y + int64_t(j) * kG);
-          if (ca * 8 < cvalid) st_cs_v4(yg + ca * 16, make_uint4(yv[0], yv[1], yv[2], yv[3]));
-          if (cb * 8 < cvalid) st_cs_v4(yg + cb * 16, make_uint4(yv[4], yv[5], yv[6], yv[7]));
-        }
-      }
-
-      // ---- row amax of d_gate (hi half) and d_up (lo half) over the 8 lanes of the row
-      uint32_t a = absmax_bf16x2(dgp[0], dgp[1]), b = absmax_bf16x2(dup[0], dup[1]);
-#pragma unroll
-      for (int c = 2; c < 8; ++c) {
-        a = absmax_bf16x2(a, dgp[c]);
-        b = absmax_bf16x2(b, dup[c]);
-      }
-      uint32_t pr = absmax_bf16x2(__byte_perm(a, b, 0x1054), __byte_perm(a, b, 0x3276));
-      pr = group_amax<kGS>(pr) & 0x7FFF7FFFu;
-
-      // ---- the row's two scales, computed by each of its 8 lanes (no shuffles
-      // on this path); lanes 0 and 1 of the row store them
-      float sg, ig, su, iu;
-      group_scale<kE4M3, kE8M0>(pr >> 16, tab, sg, ig);
-      group_scale<kE4M3, kE8M0>(pr & 0xFFFFu, tab, su, iu);
-      const int rbase = sub * kStageRows + warp * kRowsPerWarp;   // the warp's first row in the tile
-      // the first two lanes of each channel group store its d_gate / d_up
-      // scale (the d_up groups start at column gis_cols / 2)
-      {
-        constexpr int kLpg = kGS / 16;   // lanes per channel group
-        const int gl = cq & (kLpg - 1);
-        if (gl < 2 && rbase + rr < valid && (cq / kLpg) * kGS < cvalid)
-          store_scale<kE8M0>(p.gis, gis_t + (rbase + rr) * p.ld_gis + cq / kLpg +
-                                        gl * (p.gis_cols >> 1),
-                             gl ? su : sg);
-      }
-
-      // ---- quantize the row's d_gate / d_up: chunks ca and cb, 8 bytes each
-      const int r = rbase + rr;   // this lane's row within the tile
-      if (r < valid) {
-        uint4 og, ou;
-        if (__any_sync(__activemask(), ig < 0.0f || iu < 0.0f)) {   // a tiny group in this warp (rare)
-          og = (ig < 0.0f) ? quant16<kE4M3, true>(dgp, -ig, sg * kTinyPre) : quant16<kE4M3, false>(dgp, ig, sg);
-          ou = (iu < 0.0f) ? quant16<kE4M3, true>(dup, -iu, su * kTinyPre) : quant16<kE4M3, false>(dup, iu, su);
-        } else {
-          og = quant16<kE4M3, false>(dgp, ig, sg);
-          ou = quant16<kE4M3, false>(dup, iu, su);
-        }
-        int8_t* dst = giq_t + r * p.ld_giq;
-        if (ca * 8 < cvalid) {
-          st_cs_v2(dst + ca * 8, make_uint2(og.x, og.y));
-          st_cs_v2(dst + K + ca * 8, make_uint2(ou.x, ou.y));
-        }
-        if (cb * 8 < cvalid) {
-          st_cs_v2(dst + cb * 8, make_uint2(og.z, og.w));
-          st_cs_v2(dst + K + cb * 8, make_uint2(ou.z, ou.w));
+          dv[c] = *reinterpret_cast<const uint4*>(src + 2 * kBoxBytes + ch[c] * 16);
         }
       }
     }
-    if (!ok) break;
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&s.released[slot], 1) == kWarps / 2 - 1) {
+        __threadfence_block();
+        s.released[slot] = 0;
+        const uint32_t nn = n + STAGES;
+        if (nn < total) {
+          atomicMax(&s.issued, static_cast<int>(nn + 1));
+          issue_load<STAGES, kQdy>(s, &map_gate, &map_up, &map_gy, p, nn, pol);
+        }
+      }
+    }
+
+    // ---- the y buffer was last read by the column pass of tile k - kYBuf
+    if (k >= kYBuf) {
+      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_free[yb]), (k / kYBuf - 1) & 1, lim, abort_flag));
+      if (!ok) break;
+    }
+
+    // ---- math, bf16 rounding; y to the shared tile (chunks swizzled by
+    // token) and, when asked for, to global memory
+    uint32_t dgp[16], dup[16];   // chunk c: words 4c .. 4c+3
+    {
+      const int key = (r >> 4) & 7;
+      uint8_t* yrow = s.ytile[yb] + r * (kG * 2);
+      int8_t* yg = nullptr;
+      if constexpr (kY) yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + r) * p.ld_y + int64_t(j) * kG);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t yv[4];
+        const uint32_t g4[4] = {gv[c].x, gv[c].y, gv[c].z, gv[c].w};
+        const uint32_t u4[4] = {uv[c].x, uv[c].y, uv[c].z, uv[c].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (kQdy) {
+            swiglu_bwd2f(g4[e], u4[e], dq[4 * c + e], yv[e], dgp[4 * c + e], dup[4 * c + e]);
+          } else {
+            const uint32_t d4[4] = {dv[c].x, dv[c].y, dv[c].z, dv[c].w};
+            swiglu_bwd2(g4[e], u4[e], d4[e], yv[e], dgp[4 * c + e], dup[4 * c + e]);
+          }
+        }
+        const uint4 yw = make_uint4(yv[0], yv[1], yv[2], yv[3]);
+        *reinterpret_cast<uint4*>(yrow + (ch[c] ^ key) * 16) = yw;
+        if constexpr (kY) {
+          if (r < valid && ch[c] * 8 < cvalid) st_cs_v4(yg + ch[c] * 16, yw);
+        }
+      }
+    }
+
+    // ---- row amax of d_gate (hi half) and d_up (lo half) per group: over the
+    // lane's chunks of the group, then over the 4 lanes of the row
+    uint32_t pr[kNG];
+#pragma unroll
+    for (int g = 0; g < kNG; ++g) {
+      const int w0 = 4 * kSPG * g;
+      uint32_t a = absmax_bf16x2(dgp[w0], dgp[w0 + 1]), b = absmax_bf16x2(dup[w0], dup[w0 + 1]);
+#pragma unroll
+      for (int w = w0 + 2; w < w0 + 4 * kSPG; ++w) {
+        a = absmax_bf16x2(a, dgp[w]);
+        b = absmax_bf16x2(b, dup[w]);
+      }
+      uint32_t m = absmax_bf16x2(__byte_perm(a, b, 0x1054), __byte_perm(a, b, 0x3276));
+      m = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 1));
+      pr[g] = absmax_bf16x2(m, __shfl_xor_sync(kFull, m, 2)) & 0x7FFF7FFFu;
+    }
+
+    // ---- scales of the row's groups (each of its 4 lanes computes them all)
+    float sg[kNG], ig[kNG], su[kNG], iu[kNG];
+    bool tiny = false;
+#pragma unroll
+    for (int g = 0; g < kNG; ++g) {
+      group_scale<kE4M3, kE8M0>(pr[g] >> 16, tab, sg[g], ig[g]);
+      group_scale<kE4M3, kE8M0>(pr[g] & 0xFFFFu, tab, su[g], iu[g]);
+      tiny |= ig[g] < 0.0f || iu[g] < 0.0f;
+    }
+    // local group g is group gg of the tile row (the chunk order swaps the
+    // 32-channel groups of odd rows); lane 2g + t stores tensor t's scale of
+    // group g (both tensors from lane g when there are 4 groups)
+    if (r < valid) {
+      const int64_t sb = (row0 + r) * p.ld_gis + int64_t(j) * kNG;
+#pragma unroll
+      for (int g = 0; g < kNG; ++g) {
+        const int gg = kNG == 4 ? (g ^ par) : g;
+        if (gg * kGS < cvalid) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if ((kNG == 4 ? g : 2 * g + t) == q)
+              store_scale<kE8M0>(p.gis, sb + gg + t * (p.gis_cols >> 1), t ? su[g] : sg[g]);
+        }
+      }
+    }
+
+    // ---- quantize the row's d_gate / d_up: chunk c with its group's scale
+    if (r < valid) {
+      int8_t* dst = p.giq + (row0 + r) * p.ld_giq + int64_t(j) * kG;
+      if (__any_sync(__activemask(), tiny)) {   // a tiny group in this warp (rare)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int g = c / kSPG;
+          const uint2 og = ig[g] < 0.0f ? quant8<kE4M3, true>(dgp + 4 * c, -ig[g], sg[g] * kTinyPre)
+                                        : quant8<kE4M3, false>(dgp + 4 * c, ig[g], sg[g]);
+          const uint2 ou = iu[g] < 0.0f ? quant8<kE4M3, true>(dup + 4 * c, -iu[g], su[g] * kTinyPre)
+                                        : quant8<kE4M3, false>(dup + 4 * c, iu[g], su[g]);
+          if (ch[c] * 8 < cvalid) {
+            st_cs_v2(dst + ch[c] * 8, og);
+            st_cs_v2(dst + K + ch[c] * 8, ou);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int g = c / kSPG;
+          const uint2 og = quant8<kE4M3, false>(dgp + 4 * c, ig[g], sg[g]);
+          const uint2 ou = quant8<kE4M3, false>(dup + 4 * c, iu[g], su[g]);
+          if (ch[c] * 8 < cvalid) {
+            st_cs_v2(dst + ch[c] * 8, og);
+            st_cs_v2(dst + K + ch[c] * 8, ou);
+          }
+        }
+      }
+    }
     mbar_arrive(smem_u32(&s.y_ready[yb]));   // every thread: its y rows of tile k are written
 
     // ================= column pass of the previous tile
