@@ -636,13 +636,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- math, bf16 rounding; y to the shared tile (chunks swizzled by
-    // token) and, when asked for, to global memory
+    // token)
     uint32_t dgp[16], dup[16];   // chunk c: words 4c .. 4c+3
+    const int key = (r >> 4) & 7;
+    uint8_t* yrow = s.ytile[yb] + r * (kG * 2);
     {
-      const int key = (r >> 4) & 7;
-      uint8_t* yrow = s.ytile[yb] + r * (kG * 2);
-      int8_t* yg = nullptr;
-      if constexpr (kY) yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + r) * p.ld_y + int64_t(j) * kG);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t yv[4];
@@ -657,11 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             swiglu_bwd2(g4[e], u4[e], d4[e], yv[e], dgp[4 * c + e], dup[4 * c + e]);
           }
         }
-        const uint4 yw = make_uint4(yv[0], yv[1], yv[2], yv[3]);
-        *reinterpret_cast<uint4*>(yrow + (ch[c] ^ key) * 16) = yw;
-        if constexpr (kY) {
-          if (r < valid && ch[c] * 8 < cvalid) st_cs_v4(yg + ch[c] * 16, yw);
-        }
+        *reinterpret_cast<uint4*>(yrow + (ch[c] ^ key) * 16) = make_uint4(yv[0], yv[1], yv[2], yv[3]);
       }
     }
 
@@ -735,6 +729,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_cs_v2(dst + K + ch[c] * 8, ou);
           }
         }
+      }
+    }
+    // ---- y itself, bf16 (optional output), read back from the lane's own
+    // chunks of the shared tile: issued after the code stores, so the math
+    // above does not wait behind them
+    if constexpr (kY) {
+      if (r < valid) {
+        int8_t* yg = reinterpret_cast<int8_t*>(p.y) + 2 * ((row0 + r) * p.ld_y + int64_t(j) * kG);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (ch[c] * 8 < cvalid)
+            st_cs_v4(yg + ch[c] * 16, *reinterpret_cast<const uint4*>(yrow + (ch[c] ^ key) * 16));
       }
     }
     mbar_arrive(smem_u32(&s.y_ready[yb]));   // every thread: its y rows of tile k are written

@@ -164,16 +164,18 @@ def test_int8_grad_y_full_size_sampled_tiles():
     assert n_diff <= 1e-3 * total, f"{n_diff} of {total} sampled codes differ"
 
 
+@pytest.mark.parametrize("G,fmt", [(128, (0, 0, 0)), (64, (1, 0, 1)), (32, (0, 1, 0))])
 @pytest.mark.parametrize("M,K", [(1, 128), (31, 128), (127, 256), (257, 128), (640, 640)])
-def test_int8_grad_y_odd_shapes_with_y(M, K):
+def test_int8_grad_y_odd_shapes_with_y(M, K, G, fmt):
     """Tail token groups of 1..127 tokens, M % 16 != 0 (byte-wise y_q_t
-    stores), one channel tile: outputs against the oracle, y against the
-    oracle's first stage."""
+    stores), one channel tile, both variants at once (INT8 grad_y and the
+    y output) at three group sizes: outputs against the oracle, y against
+    the oracle's first stage."""
     w = W.small_workload(M, K, seed=3 * M + K, zero_group_every=5)
     x, _ = W.make_inputs(w)
     q, s = W.quantized_grad_y(w)
-    got = _run_int8_grad_y(x, q, s, 128, (0, 0, 0), pad=1, with_y=True)
-    ref = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, 128, 0, 0, 0)
-    U.compare_fmt(got[:4], ref, 0, 0, 0, f"int8 grad_y M={M} K={K}", 128)
+    got = _run_int8_grad_y(x, q, s, G, fmt, pad=1, with_y=True)
+    ref = oracle.silu_dot_fwd_bwd_quant_fuse_qgrad(x, q, s, G, *fmt)
+    U.compare_fmt(got[:4], ref, *fmt, f"int8 grad_y M={M} K={K} G={G}", G)
     U.compare_bf16(got[4], oracle.swiglu_bwd_bf16_dy(x, oracle.dequant_grad_y(q, s))[0], "y",
                    f"M={M} K={K}")
