@@ -16,16 +16,19 @@
 
 namespace {
 
-// Pipeline depth of the kernels' shared-memory rings (48 KB per stage;
-// compile-time overridable for tuning sweeps): three for the 128 x 128-tile
+// Pipeline depth of the kernels' shared-memory rings (compile-time
+// overridable for tuning sweeps): three 48 KB stages for the 128 x 128-tile
 // kernel (its two warp halves work on different slots, and a third slot
-// keeps a load in flight for each), two for the 256-group kernel (its 128 KB
-// y buffer leaves no room for a third).
+// keeps a load in flight for each), four 24 KB stages for the 256-group
+// kernel (two per warp half, next to its 128 KB y buffer).
 #ifndef SDQ_STAGES
 #define SDQ_STAGES 3
 #endif
 constexpr int kStages = SDQ_STAGES;
-constexpr int kStages256 = 2;
+#ifndef SDQ_STAGES256
+#define SDQ_STAGES256 4
+#endif
+constexpr int kStages256 = SDQ_STAGES256;
 
 constexpr int kMaxDevices = 64;
 

@@ -7,10 +7,12 @@
 // whole groups, so the work unit is a 256-token x 256-channel block, which
 // holds exactly one group on each axis:
 //
-//   * the unit arrives as eight 32-row stages of 32 x 256 elements per input
-//     (gate, up, grad_y: 48 KB a stage, the same ring protocol as the
-//     128-group kernel: mbarrier per slot, the last warp to release a slot
-//     issues its next load);
+//   * the unit arrives as sixteen 16-row stages of 16 x 256 elements per
+//     input (gate, up, grad_y: 24 KB a stage) in a 4-slot ring, with the
+//     128-group kernel's protocol (mbarrier per slot, the last warp to
+//     release a slot issues its next load); warps 0-7 take the even stages
+//     and warps 8-15 the odd ones, so each half has two slots of its own and
+//     a slot waits for 8 warps;
 //   * row pass: a lane owns 16 channels of one row (16 lanes a row, 2 rows a
 //     warp), so a whole 256-channel row group is one half-warp: its amax
 //     takes four shuffle steps and the row is quantized and stored at once;
@@ -33,13 +35,12 @@
 namespace sdq {
 
 constexpr int kG2 = 256;                             // group size = unit edge
-constexpr int kStageRows2 = 32;                      // token rows per stage
-constexpr int kStagesPerUnit = kG2 / kStageRows2;    // 8
-constexpr int kBoxBytes2 = kStageRows2 * kG2 * 2;    // one bf16 box: 16 KB
-constexpr int kStageBytes2 = 3 * kBoxBytes2;         // 48 KB
-constexpr int kQBoxBytes2 = kStageRows2 * kG2;       // one INT8 grad_y box: 8 KB
+constexpr int kStageRows2 = 16;                      // token rows per stage
+constexpr int kStagesPerUnit = kG2 / kStageRows2;    // 16
+constexpr int kBoxBytes2 = kStageRows2 * kG2 * 2;    // one bf16 box: 8 KB
+constexpr int kStageBytes2 = 3 * kBoxBytes2;         // 24 KB
+constexpr int kQBoxBytes2 = kStageRows2 * kG2;       // one INT8 grad_y box: 4 KB
 constexpr int kYBytes2 = kG2 * kG2 * 2;              // bf16 y of a unit: 128 KB
-static_assert(kStageBytes2 == kStageBytes, "both kernels use 48 KB stages");
 
 template <int STAGES>
 struct Smem256 {
@@ -59,7 +60,7 @@ constexpr size_t smem_bytes256() {
   return sizeof(Smem256<STAGES>) + 128;
 }
 
-// Load n of this CTA: stage n % 8 of its (n / 8)-th unit into slot n % STAGES.
+// Load n of this CTA: stage n % 16 of its (n / 16)-th unit into slot n % STAGES.
 template <int STAGES, bool kQdy>
 __device__ __forceinline__ void issue_load256(Smem256<STAGES>& s, const CUtensorMap* mgate,
                                               const CUtensorMap* mup, const CUtensorMap* mdy,
@@ -146,11 +147,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // row pass: lane = 16 * rr + cq owns 16-byte chunks ca, cb (8 channels
   // each) of row srow of the stage; chunks ordered so that each 8-lane
   // quarter of the warp reads 8 distinct bank groups
+  const int grp = warp >> 3;   // even (0) or odd (1) stages of every unit
   const int rr = lane >> 4;
   const int cq = lane & 15;
   const int ca = 2 * cq + ((cq >> 2) & 1);
   const int cb = 2 * cq + 1 - ((cq >> 2) & 1);
-  const int srow = warp * 2 + rr;
+  const int srow = (warp & 7) * 2 + rr;
   // column pass: thread = 8 * cp + kc, channel pairs cp and cp + 64
   const int cp0 = tid >> 3;
   const int kc = tid & 7;
@@ -198,8 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int8_t* giq_u = p.giq + row0 * p.ld_giq + j * kG2;
     const int64_t gis_u = row0 * p.ld_gis + j;
 
-    // ================= row pass over the unit's eight stages
-    for (int sub = 0; sub < kStagesPerUnit; ++sub) {
+    // ================= row pass over this half's eight stages of the unit
+    for (int sub2 = 0; sub2 < kStagesPerUnit / 2; ++sub2) {
+      const int sub = 2 * sub2 + grp;
       const uint32_t n = static_cast<uint32_t>(k) * kStagesPerUnit + sub;
       const uint32_t slot = n % STAGES;
       const int r = sub * kStageRows2 + srow;   // this lane's row within the unit
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         __threadfence_block();
-        if (atomicAdd(&s.released[slot], 1) == kWarps - 1) {
+        if (atomicAdd(&s.released[slot], 1) == kWarps / 2 - 1) {
           __threadfence_block();
           s.released[slot] = 0;
           const uint32_t nn = n + STAGES;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- y to the unit's shared tile; it was last read by the column
       // pass of the previous unit
-      if (sub == 0 && k >= 1) {
+      if (sub2 == 0 && k >= 1) {
         ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_free), (k - 1) & 1, lim, abort_flag));
         if (!ok) break;
       }
