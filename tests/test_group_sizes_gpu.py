@@ -75,9 +75,10 @@ def test_group_sizes_over_the_whole_exponent_range(G):
     _check(x, gy, G, (1, 1, 0), "exponent sweep")
 
 
-def test_group_256_on_the_outlier_workload_and_a_large_one():
-    """Groups of 256 on M=4000 K=2048 (outliers, zero groups, a 160-token tail
-    group) in full, and on M=8192 K=4096 in full, in the page's format."""
-    for idx in (3, 2):
-        x, gy = W.make_inputs(W.WORKLOADS[idx])
-        _check(x, gy, 256, (0, 0, 0), W.WORKLOADS[idx].name)
+@pytest.mark.slow
+@pytest.mark.parametrize("idx", [3, 2, 4])
+def test_group_256_on_the_outlier_and_large_workloads(idx):
+    """Groups of 256 in full, in the page's format: M=4000 K=2048 (outliers,
+    zero groups, a 160-token tail group), M=8192 K=4096 and M=16384 K=7168."""
+    x, gy = W.make_inputs(W.WORKLOADS[idx])
+    _check(x, gy, 256, (0, 0, 0), W.WORKLOADS[idx].name)
