@@ -10,7 +10,8 @@ case and the largest of the five workloads).  Prints ONE JSON line on rank 0;
 besides the headline it carries a per_workload list timing all five
 workloads (skipped with --no-per-workload).
 
-Timing: W eager warm-up calls, then EXACTLY K calls replayed from CUDA
+Timing: W untimed warm-up calls (one eager, W-1 replayed from a CUDA graph
+just before the timed region), then EXACTLY K calls replayed from CUDA
 graphs, bracketed by a barrier and a device synchronize and timed with CUDA
 events on the launching stream; the maximum over ranks is taken.  Between
 consecutive calls the inputs and outputs rotate through enough buffer sets to
@@ -282,6 +283,9 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = pick_workload(args.workload)
+    if args.group_size != w.group_size:   # same inputs, another group size
+        w = W.Workload(w.name, w.M, w.K, w.sigma_x, w.sigma_grad_y, w.seed, args.group_size,
+                       w.outlier_frac, w.outlier_mult, w.zero_group_every)
     x, gy = W.make_inputs(w)
     import oracle
     G = w.group_size
@@ -291,7 +295,7 @@ def run_reference(args):
         i = s % Mg
         r0, r1 = i * G, min(w.M, i * G + G)
         oracle.silu_dot_fwd_bwd_quant_fuse(x[r0:r1], gy[r0:r1], G)
-        return W.Workload("s", r1 - r0, w.K, 1, 1, 0).algorithmic_bytes()
+        return W.Workload("s", r1 - r0, w.K, 1, 1, 0, G).algorithmic_bytes()
 
     for s in range(args.warmup):
         step(s)
@@ -306,10 +310,10 @@ def run_reference(args):
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, None, args.gpus),
-        "step": "one 128-token group x all K channels of the workload (a bounded sample), "
+        "step": f"one {G}-token group x all K channels of the workload (a bounded sample), "
                 "cycling through its token groups",
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} steps of one 128-token group x K={w.K}"},
+                         "sample": f"{args.steps} steps of one {G}-token group x K={w.K}"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -371,22 +375,31 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
         sdq.silu_dot_fwd_bwd_quant_fuse(xs, gs, *outs, w.group_size, codes=codes, scales=scales,
                                         y_scale_layout=layout, y=ys, grad_y_s=gss)
 
-    for k in range(warmup):
-        call(k)
+    # W untimed warm-up calls: the first eager (it sets up the library on the
+    # device), the other W-1 replayed from a graph right before the timed
+    # region, so the GPU is not left idle while the graphs are captured.
+    call(0)
     torch.cuda.synchronize(device)
-    # Capture the K timed calls into CUDA graphs (chunks of at most 1000 calls).
-    chunk = min(steps, 1000)
-    graphs = []
-    done = 0
-    while done < steps:
-        n = min(chunk, steps - done)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
-            for k in range(n):
-                call(warmup + done + k)
-        graphs.append(g)
-        done += n
+
+    def capture(first: int, count: int):
+        """CUDA graphs of `count` calls from call index `first` (chunks of at most 1000)."""
+        out, done = [], 0
+        while done < count:
+            n = min(1000, count - done)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+                for k in range(n):
+                    call(first + done + k)
+            out.append(g)
+            done += n
+        return out
+
+    warm = capture(1, warmup - 1)
+    graphs = capture(warmup, steps)
     from swiglu_backward_int8_b200 import parallel
+    torch.cuda.synchronize(device)
+    for g in warm:
+        g.replay()
     torch.cuda.synchronize(device)
     parallel.barrier(device)
     torch.cuda.synchronize(device)
@@ -403,7 +416,7 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
     st = sdq.sdq_device_status(stream.cuda_stream)
     if st != 0:
         raise RuntimeError(f"device status {sdq.status_string(st)}")
-    del graphs
+    del graphs, warm
     return ms, (t0, t1), nsets
 
 
@@ -620,22 +633,30 @@ def run_fwd(args):
         xs, wt, h, q8 = sets[k % nsets]
         sdq.swiglu_q8_1(xs[:, :inter], xs[:, inter:], wt, args.limit, h, q8)
 
-    for k in range(args.warmup):
-        call(k)
+    call(0)   # warm-up 1 of W, eager: sets the library up on the device
     torch.cuda.synchronize(device)
-    graphs, done = [], 0
-    while done < args.steps:
-        n = min(1000, args.steps - done)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
-            for k in range(n):
-                call(args.warmup + done + k)
-        graphs.append(g)
-        done += n
+
+    def capture(first: int, count: int):
+        out, done = [], 0
+        while done < count:
+            n = min(1000, count - done)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+                for k in range(n):
+                    call(first + done + k)
+            out.append(g)
+            done += n
+        return out
+
+    warm = capture(1, args.warmup - 1)   # warm-up 2..W, replayed right before the timed region
+    graphs = capture(args.warmup, args.steps)
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     time.sleep(0.3)
     stream = torch.cuda.current_stream(device)
+    for g in warm:
+        g.replay()
+    torch.cuda.synchronize(device)
     parallel.barrier(device)
     torch.cuda.synchronize(device)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -686,7 +707,7 @@ def run_fwd(args):
             "e2e": {"unavailable": "the forward op has a device entry point only"},
             "gpu_launches": args.steps, "clocks": clocks, "kernel_sources_sha": kernel_sha(FWD_SOURCES),
         }), flush=True)
-    del graphs
+    del graphs, warm
     import torch.distributed as tdist
     if tdist.is_initialized():
         parallel.barrier(device)

@@ -21,8 +21,10 @@
 //     256 tokens (a thread takes 2 channels x 32 tokens, twice; 8 threads
 //     share a column group);
 //   * there is one y buffer (two would not fit next to the ring), so a
-//     unit's row pass waits until every thread has finished the column pass
-//     of the unit before; the ring keeps loading meanwhile.
+//     unit's row pass waits until every thread has read its column words of
+//     the unit before (each thread holds its 64 words in registers and hands
+//     the tile back before its column arithmetic); the ring keeps loading
+//     meanwhile.
 //
 // Rows past M and channels past K are zero-filled by the TMA unit; zeros
 // never change an amax, and their outputs are not stored, so a tail token
@@ -87,16 +89,20 @@ __device__ __forceinline__ int y256_off(int tok, int c) {
 }
 
 // Column pass of one task: channels 2cp, 2cp+1 and tokens 32kc .. 32kc+31 of
-// the unit; the column amax over the 8 threads (kc = 0..7) that share the
-// channels, the two scales, codes, four 16-byte pieces of y_q_t rows.
-template <bool kE4M3, bool kE8M0, bool kYsMgK>
-__device__ __forceinline__ void column_pass256(const uint8_t* yt, const float2* tab, const Params& p,
-                                               int i, int j, int64_t row0, int valid, int cp, int kc) {
-  constexpr unsigned kFull = 0xffffffffu;
-  uint32_t v[32];
+// the unit, in two parts: the words are read from the y tile first (so the
+// tile can be handed back before the arithmetic), then the column amax over
+// the 8 threads (kc = 0..7) that share the channels, the two scales, codes,
+// four 16-byte pieces of y_q_t rows.
+__device__ __forceinline__ void column_load256(const uint8_t* yt, int cp, int kc, uint32_t (&v)[32]) {
 #pragma unroll
   for (int tt = 0; tt < 32; ++tt)
     v[tt] = *reinterpret_cast<const uint32_t*>(yt + y256_off(32 * kc + tt, cp >> 2) + ((cp & 3) << 2));
+}
+
+template <bool kE4M3, bool kE8M0, bool kYsMgK>
+__device__ __forceinline__ void column_quant256(const uint32_t (&v)[32], const float2* tab, const Params& p,
+                                                int i, int j, int64_t row0, int valid, int cp, int kc) {
+  constexpr unsigned kFull = 0xffffffffu;
   uint32_t m = absmax_bf16x2(v[0], v[1]);
 #pragma unroll
   for (int tt = 2; tt < 32; ++tt) m = absmax_bf16x2(m, v[tt]);
@@ -107,7 +113,7 @@ __device__ __forceinline__ void column_pass256(const uint8_t* yt, const float2* 
   group_scale<kE4M3, kE8M0>(m & 0xFFFFu, tab, s_lo, i_lo);
   group_scale<kE4M3, kE8M0>(m >> 16, tab, s_hi, i_hi);
   const int ch = j * kG2 + 2 * cp;
-  const bool ch_ok = ch < p.K;   // a partial last unit's missing channels are zeros, not stored
+  const bool ch_ok = ch < p.K;
   if (kc < 2 && ch_ok)
     store_scale<kE8M0>(p.yst, kYsMgK ? int64_t(i) * p.ld_yst + ch + kc : int64_t(ch + kc) * p.ld_yst + i,
                        kc ? s_hi : s_lo);
@@ -316,9 +322,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================= column pass of this unit: channel pairs cp0 and cp0 + 64
     ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.y_ready), k & 1, lim, abort_flag));
     if (!ok) break;
-    column_pass256<kE4M3, kE8M0, kYsMgK>(s.ytile, tab, p, i, j, row0, valid, cp0, kc);
-    column_pass256<kE4M3, kE8M0, kYsMgK>(s.ytile, tab, p, i, j, row0, valid, cp0 + 64, kc);
-    mbar_arrive(smem_u32(&s.y_free));
+    {
+      uint32_t va[32], vb[32];
+      column_load256(s.ytile, cp0, kc, va);
+      column_load256(s.ytile, cp0 + 64, kc, vb);
+      mbar_arrive(smem_u32(&s.y_free));   // the tile's words are in registers: it may be rewritten
+      column_quant256<kE4M3, kE8M0, kYsMgK>(va, tab, p, i, j, row0, valid, cp0, kc);
+      column_quant256<kE4M3, kE8M0, kYsMgK>(vb, tab, p, i, j, row0, valid, cp0 + 64, kc);
+    }
   }
 
   __syncthreads();
