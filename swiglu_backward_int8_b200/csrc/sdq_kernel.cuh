@@ -10,7 +10,8 @@
 // Template variants (each its own instantiation, so a variant's work never
 // reaches the others): group size 128, 64 or 32 (a tile holds whole groups
 // of each); code format INT8 or FP8 E4M3, scale format fp32 or E8M0, y_s_t
-// [K, Mg] or [Mg, K]; kY, the recomputed bf16 y also stored from registers;
+// [K, Mg] or [Mg, K]; kY, the recomputed bf16 y also stored (read back from
+// the shared y tile after the code stores);
 // kQdy, grad_y read as INT8 codes (an 8-bit box in the stage's third slot)
 // times one fp32 scale per token and 128 channels.
 //
@@ -30,6 +31,9 @@
 //     warp, so every warp computes and may use 128 registers.
 //     Rows past M are zero-filled by the TMA unit, and zeros never change an
 //     amax, so a tail token group is quantized over exactly the tokens it holds.
+//     With an odd STAGES a slot's consecutive loads belong to different warp
+//     halves (below), so a half waits for the slot's previous load before it
+//     waits on the parity of its own.
 //   * row pass: warps 0-7 take the first stage of every tile and warps 8-15
 //     the second, so the two halves of the CTA work on different slots and a
 //     slot waits for 8 warps, not 16.  A lane owns 32 channels of one token
@@ -594,6 +598,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     float dsc = 0.0f;   // INT8 grad_y: the scale of this lane's row in tile column j
     if constexpr (kQdy) {
       if (r < valid) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + j);
+    }
+    // With an odd STAGES a slot's consecutive loads n - STAGES and n go to
+    // different warp halves, and a half may run a tile ahead of the other: if
+    // load n - STAGES has not landed yet, a wait on n's parity alone would
+    // match the slot's phase before it and return at once.  So the half first
+    // waits for load n - STAGES (that wait can only match it: load n - 2 STAGES
+    // was this half's own, and load n is not issued before n - STAGES is
+    // released); with an even STAGES it returns at once.
+    if (n >= STAGES) {
+      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES - 1) & 1u, lim, abort_flag));
+      if (!ok) break;
     }
     ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
     if (!ok) break;

@@ -216,6 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kQdy) {   // INT8 grad_y: its scale per token and 128 channels
         if (r < valid && j * kG2 + 16 * cq < K) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + 2 * j + (cq >> 3));
       }
+      // (an odd STAGES would hand a slot's consecutive loads to different
+      // halves: then wait for the slot's previous load first, as in the
+      // 128-group kernel; with the even ring here it returns at once)
+      if (STAGES % 2 == 1 && n >= STAGES) {
+        ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES - 1) & 1u, lim, abort_flag));
+        if (!ok) break;
+      }
       ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
       if (!ok) break;
 

@@ -300,3 +300,32 @@ def test_concurrent_streams_and_graph_replay_are_bit_identical():
                 assert torch.equal(a.cpu(), b)
     assert sdq.sdq_device_status() == 0
     del g
+
+
+def test_back_to_back_bursts_are_bit_identical():
+    """Stress for the shared-memory ring: 25 bursts of 8 back-to-back calls
+    (each into its own outputs, so consecutive launches overlap their start
+    and end) on M=8192 K=4096, every call's four outputs compared byte for
+    byte with a single call's, and that call with the oracle.  A stage read
+    before its copy had landed would show as a difference."""
+    import swiglu_backward_int8_b200 as sdq
+    w = W.WORKLOADS[2]
+    x, gy = W.make_inputs(w)
+    xd, gyd = U.to_device_bf16(x), U.to_device_bf16(gy)
+    ref = sdq.allocate_outputs(w.M, w.K, "cuda")
+    sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *ref)
+    torch.cuda.synchronize()
+    U.compare([t.cpu().numpy() for t in ref], oracle.silu_dot_fwd_bwd_quant_fuse(x, gy), w.name)
+    sets = [sdq.allocate_outputs(w.M, w.K, "cuda") for _ in range(8)]
+    bad = 0
+    for _ in range(25):
+        for o in sets:
+            for t in o:
+                t.zero_()
+        for o in sets:
+            sdq.silu_dot_fwd_bwd_quant_fuse(xd, gyd, *o)
+        for o in sets:
+            bad += sum(int(not torch.equal(a, b)) for a, b in zip(o, ref))
+    torch.cuda.synchronize()
+    assert sdq.sdq_device_status() == 0
+    assert bad == 0, f"{bad} outputs differ from a single call's"
