@@ -31,9 +31,9 @@
 //     warp, so every warp computes and may use 128 registers.
 //     Rows past M are zero-filled by the TMA unit, and zeros never change an
 //     amax, so a tail token group is quantized over exactly the tokens it holds.
-//     With an odd STAGES a slot's consecutive loads belong to different warp
-//     halves (below), so a half waits for the slot's previous load before it
-//     waits on the parity of its own.
+//     Each slot has two mbarriers that take its loads in turn, so that with
+//     an odd STAGES (consecutive loads of a slot going to different warp
+//     halves, below) every barrier's uses still belong to one half.
 //   * row pass: warps 0-7 take the first stage of every tile and warps 8-15
 //     the second, so the two halves of the CTA work on different slots and a
 //     slot waits for 8 warps, not 16.  A lane owns 32 channels of one token
@@ -123,7 +123,7 @@ struct Smem {
   alignas(128) uint8_t ring[STAGES][kStageBytes];  // [gate | up | grad_y], each [64][128] bf16
   alignas(16) uint8_t ytile[kYBuf][kYBytes];       // bf16 y [token][channel], chunks swizzled
   alignas(16) float2 scale_tab[128];               // per bf16 mantissa m: scale and inverse for 2^0 (see group_scale)
-  alignas(8) uint64_t full[STAGES];
+  alignas(8) uint64_t full[STAGES][2];             // per slot, alternate loads (ring_bar_index)
   alignas(8) uint64_t y_ready[kYBuf];              // all threads wrote their rows of the y tile
   alignas(8) uint64_t y_free[kYBuf];               // all threads finished reading the y tile
   int released[STAGES];                            // warps done with the slot's current load
@@ -134,6 +134,21 @@ struct Smem {
 template <int STAGES>
 constexpr size_t smem_bytes() {
   return sizeof(Smem<STAGES>) + 128;  // + room to align the base to 128 B
+}
+
+// The ring barrier of load n and the parity a consumer waits on.  Each slot
+// has two barriers that take its loads in turn, so consecutive uses of one
+// barrier are loads n and n + 2 STAGES.  The two warp halves take alternate
+// loads, so those are always the same half's, consumed in order: when a half
+// waits on load n's barrier, the barrier is in load n's phase or just past it,
+// never a phase behind (with one barrier per slot and an odd STAGES, a half
+// that ran a tile ahead could find the slot a phase behind, with the same
+// parity as the one it waits for, and read the slot before its copy landed).
+__device__ __forceinline__ uint32_t ring_bar_index(uint32_t n, uint32_t stages) {
+  return 2 * (n % stages) + ((n / stages) & 1u);
+}
+__device__ __forceinline__ uint32_t ring_parity(uint32_t n, uint32_t stages) {
+  return (n / (2 * stages)) & 1u;
 }
 
 // Tile t -> (token-group i, channel-group j), banded: kTileBand tile rows per
@@ -168,7 +183,7 @@ __device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* m
   tile_ij(t, p.Mg, p.Kg, i, j);
   const int r = i * kG + static_cast<int>(n % kStagesPerTile) * kStageRows;
   const uint32_t slot = n % STAGES;
-  const uint32_t fb = smem_u32(&s.full[slot]);
+  const uint32_t fb = smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES));
   mbar_arrive_expect_tx(fb, kQdy ? 2 * kBoxBytes + kQBoxBytes : kStageBytes);
   const uint32_t dst = smem_u32(s.ring[slot]);
   tma_load_2d(dst, mgate, fb, j * kG, r, pol);
@@ -547,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&map_up);
     prefetch_tensormap(&map_gy);
     for (int st = 0; st < STAGES; ++st) {
-      mbar_init(smem_u32(&s.full[st]), 1);
+      mbar_init(smem_u32(&s.full[st][0]), 1);
+      mbar_init(smem_u32(&s.full[st][1]), 1);
       s.released[st] = 0;
     }
     for (int b = 0; b < kYBuf; ++b) {
@@ -599,18 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (kQdy) {
       if (r < valid) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + j);
     }
-    // With an odd STAGES a slot's consecutive loads n - STAGES and n go to
-    // different warp halves, and a half may run a tile ahead of the other: if
-    // load n - STAGES has not landed yet, a wait on n's parity alone would
-    // match the slot's phase before it and return at once.  So the half first
-    // waits for load n - STAGES (that wait can only match it: load n - 2 STAGES
-    // was this half's own, and load n is not issued before n - STAGES is
-    // released); with an even STAGES it returns at once.
-    if (n >= STAGES) {
-      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES - 1) & 1u, lim, abort_flag));
-      if (!ok) break;
-    }
-    ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
+    ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES)),
+                                         ring_parity(n, STAGES), lim, abort_flag));
     if (!ok) break;
 
     // ---- stage -> registers, then release the slot (the last of the 8 warps refills it)
@@ -790,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t issued = static_cast<uint32_t>(s.issued);
     const uint32_t first = issued > STAGES ? issued - STAGES : 0;
     for (uint32_t n = first; n < issued; ++n)
-      mbar_wait(smem_u32(&s.full[n % STAGES]), (n / STAGES) & 1u, lim);
+      mbar_wait(smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES)), ring_parity(n, STAGES), lim);
   }
 }
 

@@ -49,7 +49,7 @@ struct Smem256 {
   alignas(128) uint8_t ring[STAGES][kStageBytes2];
   alignas(16) uint8_t ytile[kYBytes2];               // [token][channel], 16-byte chunks swizzled
   alignas(16) float2 scale_tab[128];
-  alignas(8) uint64_t full[STAGES];
+  alignas(8) uint64_t full[STAGES][2];               // per slot, alternate loads (ring_bar_index)
   alignas(8) uint64_t y_ready;                       // every thread wrote its y rows of the unit
   alignas(8) uint64_t y_free;                        // every thread finished the unit's column pass
   int released[STAGES];
@@ -72,7 +72,7 @@ __device__ __forceinline__ void issue_load256(Smem256<STAGES>& s, const CUtensor
   tile_ij(t, p.Mg, p.Kg, i, j);
   const int r = i * kG2 + static_cast<int>(n % kStagesPerUnit) * kStageRows2;
   const uint32_t slot = n % STAGES;
-  const uint32_t fb = smem_u32(&s.full[slot]);
+  const uint32_t fb = smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES));
   mbar_arrive_expect_tx(fb, kQdy ? 2 * kBoxBytes2 + kQBoxBytes2 : kStageBytes2);
   const uint32_t dst = smem_u32(s.ring[slot]);
   tma_load_2d(dst, mgate, fb, j * kG2, r, pol);
@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&map_up);
     prefetch_tensormap(&map_gy);
     for (int st = 0; st < STAGES; ++st) {
-      mbar_init(smem_u32(&s.full[st]), 1);
+      mbar_init(smem_u32(&s.full[st][0]), 1);
+      mbar_init(smem_u32(&s.full[st][1]), 1);
       s.released[st] = 0;
     }
     mbar_init(smem_u32(&s.y_ready), kThreads);
@@ -216,14 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kQdy) {   // INT8 grad_y: its scale per token and 128 channels
         if (r < valid && j * kG2 + 16 * cq < K) dsc = __ldg(p.gys + (row0 + r) * p.ld_gys + 2 * j + (cq >> 3));
       }
-      // (an odd STAGES would hand a slot's consecutive loads to different
-      // halves: then wait for the slot's previous load first, as in the
-      // 128-group kernel; with the even ring here it returns at once)
-      if (STAGES % 2 == 1 && n >= STAGES) {
-        ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES - 1) & 1u, lim, abort_flag));
-        if (!ok) break;
-      }
-      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[slot]), (n / STAGES) & 1u, lim, abort_flag));
+      ok = __all_sync(kFull, wait_or_abort(smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES)),
+                                           ring_parity(n, STAGES), lim, abort_flag));
       if (!ok) break;
 
       uint32_t gw[8], uw[8], dw[8];
@@ -344,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t issued = static_cast<uint32_t>(s.issued);
     const uint32_t first = issued > STAGES ? issued - STAGES : 0;
     for (uint32_t n = first; n < issued; ++n)
-      mbar_wait(smem_u32(&s.full[n % STAGES]), (n / STAGES) & 1u, lim);
+      mbar_wait(smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES)), ring_parity(n, STAGES), lim);
   }
 }
 

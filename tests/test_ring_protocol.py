@@ -1,0 +1,116 @@
+"""A discrete-event model of the fused kernel's shared-memory ring, checked on
+the CPU.
+
+The 128-tile kernel keeps STAGES slots; load n goes into slot n % STAGES and
+is consumed by the warp half n % 2 (8 warps); the last warp of the half to
+release a slot issues load n + STAGES into it.  A consumer waits on an
+mbarrier with a parity, and the hardware only compares parities: a parity
+wait succeeds when the barrier's current phase has the other parity.  The
+model reproduces that rule exactly and drives the protocol with random load
+latencies and compute times (one half may run a tile ahead of the other).
+
+It checks two designs of the barriers:
+  * one barrier per slot, waited on with parity (n / STAGES) % 2: with an
+    odd STAGES a slot's consecutive loads belong to different halves, and a
+    half that ran ahead finds the barrier one phase behind with the parity of
+    an older, completed phase -- it reads the slot before its copy landed;
+  * two barriers per slot taking its loads in turn (load n on barrier
+    2 (n % STAGES) + (n / STAGES) % 2, parity (n / (2 STAGES)) % 2), the
+    kernel's design: consecutive uses of a barrier are loads n and
+    n + 2 STAGES, always the same half's, so no wait can match an older phase.
+"""
+from __future__ import annotations
+
+import random
+
+import pytest
+
+
+def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed: int = 0):
+    """Returns (finished, early_reads)."""
+    rng = random.Random(seed)
+    nbar = stages * (2 if two_barriers else 1)
+    phase = [0] * nbar          # current phase of each barrier
+    pending = [0] * nbar        # copies outstanding in the current phase
+    armed = [False] * nbar      # the phase's one arrival (with its byte count) happened
+    content = [None] * stages   # load whose data sits in the slot
+    released = [0] * stages
+    total = 2 * tiles
+    in_flight = []              # (land time, load)
+
+    def bar(n):
+        return 2 * (n % stages) + ((n // stages) & 1) if two_barriers else n % stages
+
+    def parity(n):
+        return (n // (2 * stages)) & 1 if two_barriers else (n // stages) & 1
+
+    def issue(n, now):
+        b = bar(n)
+        armed[b] = True
+        pending[b] += 1
+        content[n % stages] = None
+        in_flight.append((now + rng.uniform(1.0, 3.0), n))
+
+    for n in range(min(stages, total)):
+        issue(n, 0.0)
+    warp_state = [{"half": w // warps, "tile": 0, "ready": 0.0} for w in range(2 * warps)]
+    early = 0
+    now = 0.0
+    for _ in range(100000):
+        moved = False
+        for w in warp_state:
+            if w["tile"] >= tiles or w["ready"] > now:
+                continue
+            n = 2 * w["tile"] + w["half"]
+            if (phase[bar(n)] & 1) == parity(n):
+                continue                      # the parity wait is still blocked
+            slot = n % stages
+            if content[slot] != n:
+                early += 1                    # read before its own copy landed
+            released[slot] += 1
+            if released[slot] == warps:       # the last of the half refills the slot
+                released[slot] = 0
+                if n + stages < total:
+                    issue(n + stages, now)
+            w["tile"] += 1
+            w["ready"] = now + rng.uniform(0.5, 4.0)
+            moved = True
+        if all(w["tile"] >= tiles for w in warp_state):
+            return True, early
+        if moved:
+            continue
+        times = [t for t, _ in in_flight] + [w["ready"] for w in warp_state
+                                             if w["tile"] < tiles and w["ready"] > now]
+        if not times:
+            return False, early               # nothing can move: deadlock
+        now = min(times)
+        for t, n in sorted(e for e in in_flight if e[0] <= now):
+            in_flight.remove((t, n))
+            b = bar(n)
+            pending[b] -= 1
+            content[n % stages] = n
+            if pending[b] == 0 and armed[b]:
+                phase[b] += 1
+                armed[b] = False
+    return False, early
+
+
+@pytest.mark.parametrize("stages", [2, 3, 4, 5])
+def test_two_barriers_per_slot_never_read_early(stages):
+    for seed in range(60):
+        finished, early = _run(True, stages, seed=seed)
+        assert finished and early == 0, (stages, seed, finished, early)
+
+
+def test_one_barrier_per_slot_reads_early_with_three_slots():
+    """The model catches the race the kernel had with one barrier per slot."""
+    bad = sum(_run(False, 3, seed=seed)[1] > 0 for seed in range(60))
+    assert bad > 0
+
+
+def test_one_barrier_per_slot_is_safe_with_an_even_ring():
+    """With an even ring each slot's loads all belong to one half (the
+    256-group kernel's 4 slots), so one barrier per slot would do there."""
+    for seed in range(60):
+        finished, early = _run(False, 4, seed=seed)
+        assert finished and early == 0, (seed, finished, early)
