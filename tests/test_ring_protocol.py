@@ -26,8 +26,10 @@ import random
 import pytest
 
 
-def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed: int = 0):
-    """Returns (finished, early_reads)."""
+def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed: int = 0,
+         groups: int = 2):
+    """`groups` warp groups of `warps` warps each take loads in turn (the
+    kernel: 2 groups of 8).  Returns (finished, early_reads)."""
     rng = random.Random(seed)
     nbar = stages * (2 if two_barriers else 1)
     phase = [0] * nbar          # current phase of each barrier
@@ -35,7 +37,7 @@ def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed:
     armed = [False] * nbar      # the phase's one arrival (with its byte count) happened
     content = [None] * stages   # load whose data sits in the slot
     released = [0] * stages
-    total = 2 * tiles
+    total = groups * tiles
     in_flight = []              # (land time, load)
 
     def bar(n):
@@ -53,7 +55,7 @@ def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed:
 
     for n in range(min(stages, total)):
         issue(n, 0.0)
-    warp_state = [{"half": w // warps, "tile": 0, "ready": 0.0} for w in range(2 * warps)]
+    warp_state = [{"half": w // warps, "tile": 0, "ready": 0.0} for w in range(groups * warps)]
     early = 0
     now = 0.0
     for _ in range(100000):
@@ -61,7 +63,7 @@ def _run(two_barriers: bool, stages: int, tiles: int = 30, warps: int = 8, seed:
         for w in warp_state:
             if w["tile"] >= tiles or w["ready"] > now:
                 continue
-            n = 2 * w["tile"] + w["half"]
+            n = groups * w["tile"] + w["half"]
             if (phase[bar(n)] & 1) == parity(n):
                 continue                      # the parity wait is still blocked
             slot = n % stages
@@ -114,3 +116,13 @@ def test_one_barrier_per_slot_is_safe_with_an_even_ring():
     for seed in range(60):
         finished, early = _run(False, 4, seed=seed)
         assert finished and early == 0, (seed, finished, early)
+
+
+@pytest.mark.parametrize("groups,stages", [(4, 6), (8, 12), (4, 4)])
+def test_two_barriers_per_slot_with_more_groups(groups, stages):
+    """More, smaller stages per tile (a layout that was measured and not
+    kept): safe whenever 2 * stages is a multiple of the group count, since
+    a barrier's consecutive loads n and n + 2 * stages then share a group."""
+    for seed in range(40):
+        finished, early = _run(True, stages, warps=16 // groups, seed=seed, groups=groups)
+        assert finished and early == 0, (groups, stages, seed, finished, early)
