@@ -53,6 +53,12 @@
 //     share its channels, computes the two column scales, quantizes its 32 y
 //     values and stores two 16-byte pieces of y_q_t rows; each group of 8
 //     threads writes one 128-byte line.
+//   * launch: the kernel is launched with programmatic stream serialization
+//     and allows the next grid to launch at once, so a CTA starts as soon as
+//     the previous grid's CTA on its SM exits, and waits (griddepcontrol) for
+//     the whole previous grid before it loads.  Meanwhile it prefetches the
+//     boxes of its first STAGES loads into L2, so they land from L2 after the
+//     wait instead of taking a DRAM round trip.
 //   * shared-memory layouts are chosen for conflict-free access: a lane of an
 //     odd row takes its chunks in the order (4k + q) ^ 4, so each 8-lane
 //     quarter of a warp reads 8 distinct bank groups, and the y tile's chunks
@@ -171,6 +177,15 @@ __device__ __forceinline__ void tile_ij(int t, int Mg, int Kg, int& i, int& j) {
   }
 }
 
+// Tensor coordinates (channel x, token y) of the boxes of load n of this CTA.
+__device__ __forceinline__ void load_coords(const Params& p, uint32_t n, int& x, int& y) {
+  const int t = blockIdx.x + static_cast<int>(n / kStagesPerTile) * gridDim.x;
+  int i, j;
+  tile_ij(t, p.Mg, p.Kg, i, j);
+  x = j * kG;
+  y = i * kG + static_cast<int>(n % kStagesPerTile) * kStageRows;
+}
+
 // Load n of this CTA: stage n % 2 of its (n / 2)-th tile, into slot n % STAGES.
 // The three input tensor maps (gate, up, grad_y: [M, K] bf16 each, with their
 // own row strides; gate and up may be the two halves of one x = [gate | up]).
@@ -178,17 +193,15 @@ template <int STAGES, bool kQdy>
 __device__ __forceinline__ void issue_load(Smem<STAGES>& s, const CUtensorMap* mgate,
                                            const CUtensorMap* mup, const CUtensorMap* mdy,
                                            const Params& p, uint32_t n, uint64_t pol) {
-  const int t = blockIdx.x + static_cast<int>(n / kStagesPerTile) * gridDim.x;
-  int i, j;
-  tile_ij(t, p.Mg, p.Kg, i, j);
-  const int r = i * kG + static_cast<int>(n % kStagesPerTile) * kStageRows;
+  int x, r;
+  load_coords(p, n, x, r);
   const uint32_t slot = n % STAGES;
   const uint32_t fb = smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES));
   mbar_arrive_expect_tx(fb, kQdy ? 2 * kBoxBytes + kQBoxBytes : kStageBytes);
   const uint32_t dst = smem_u32(s.ring[slot]);
-  tma_load_2d(dst, mgate, fb, j * kG, r, pol);
-  tma_load_2d(dst + kBoxBytes, mup, fb, j * kG, r, pol);
-  tma_load_2d(dst + 2 * kBoxBytes, mdy, fb, j * kG, r, pol);
+  tma_load_2d(dst, mgate, fb, x, r, pol);
+  tma_load_2d(dst + kBoxBytes, mup, fb, x, r, pol);
+  tma_load_2d(dst + 2 * kBoxBytes, mdy, fb, x, r, pol);
 }
 
 // bf16 pair -> two floats (exact).
@@ -572,8 +585,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     s.abort = 0;
     fence_mbar_init();
-    grid_dependency_wait();   // inputs may come from the previous kernel in the stream
+    // While the previous grid of the stream finishes (this CTA can start as
+    // soon as its SM is free), warm L2 with the boxes of the first loads:
+    // they then land from L2 right after the wait instead of from DRAM.
     const uint32_t first = total < STAGES ? total : STAGES;
+    for (uint32_t n = 0; n < first; ++n) {
+      int x, y;
+      load_coords(p, n, x, y);
+      tma_prefetch_l2_2d(&map_gate, x, y);
+      tma_prefetch_l2_2d(&map_up, x, y);
+      tma_prefetch_l2_2d(&map_gy, x, y);
+    }
+    grid_dependency_wait();   // inputs may come from the previous kernel in the stream
     s.issued = static_cast<int>(first);
     for (uint32_t n = 0; n < first; ++n)
       if (n != 0 || !p.withhold_first_load)

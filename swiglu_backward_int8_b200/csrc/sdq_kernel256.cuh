@@ -62,22 +62,29 @@ constexpr size_t smem_bytes256() {
   return sizeof(Smem256<STAGES>) + 128;
 }
 
+// Tensor coordinates (channel x, token y) of the boxes of load n of this CTA.
+__device__ __forceinline__ void load_coords256(const Params& p, uint32_t n, int& x, int& y) {
+  const int t = blockIdx.x + static_cast<int>(n / kStagesPerUnit) * gridDim.x;
+  int i, j;
+  tile_ij(t, p.Mg, p.Kg, i, j);
+  x = j * kG2;
+  y = i * kG2 + static_cast<int>(n % kStagesPerUnit) * kStageRows2;
+}
+
 // Load n of this CTA: stage n % 16 of its (n / 16)-th unit into slot n % STAGES.
 template <int STAGES, bool kQdy>
 __device__ __forceinline__ void issue_load256(Smem256<STAGES>& s, const CUtensorMap* mgate,
                                               const CUtensorMap* mup, const CUtensorMap* mdy,
                                               const Params& p, uint32_t n, uint64_t pol) {
-  const int t = blockIdx.x + static_cast<int>(n / kStagesPerUnit) * gridDim.x;
-  int i, j;
-  tile_ij(t, p.Mg, p.Kg, i, j);
-  const int r = i * kG2 + static_cast<int>(n % kStagesPerUnit) * kStageRows2;
+  int x, r;
+  load_coords256(p, n, x, r);
   const uint32_t slot = n % STAGES;
   const uint32_t fb = smem_u32(&s.full[0][0] + ring_bar_index(n, STAGES));
   mbar_arrive_expect_tx(fb, kQdy ? 2 * kBoxBytes2 + kQBoxBytes2 : kStageBytes2);
   const uint32_t dst = smem_u32(s.ring[slot]);
-  tma_load_2d(dst, mgate, fb, j * kG2, r, pol);
-  tma_load_2d(dst + kBoxBytes2, mup, fb, j * kG2, r, pol);
-  tma_load_2d(dst + 2 * kBoxBytes2, mdy, fb, j * kG2, r, pol);
+  tma_load_2d(dst, mgate, fb, x, r, pol);
+  tma_load_2d(dst + kBoxBytes2, mup, fb, x, r, pol);
+  tma_load_2d(dst + 2 * kBoxBytes2, mdy, fb, x, r, pol);
 }
 
 // Byte offset of 16-byte chunk c (0..31) of token row `tok` in the y tile:
@@ -180,8 +187,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&s.y_free), kThreads);
     s.abort = 0;
     fence_mbar_init();
-    grid_dependency_wait();
+    // L2 prefetch of the first loads' boxes while the previous grid finishes
+    // (as in the 128-group kernel)
     const uint32_t first = total < STAGES ? total : STAGES;
+    for (uint32_t n = 0; n < first; ++n) {
+      int x, y;
+      load_coords256(p, n, x, y);
+      tma_prefetch_l2_2d(&map_gate, x, y);
+      tma_prefetch_l2_2d(&map_up, x, y);
+      tma_prefetch_l2_2d(&map_gy, x, y);
+    }
+    grid_dependency_wait();
     s.issued = static_cast<int>(first);
     for (uint32_t n = 0; n < first; ++n)
       if (n != 0 || !p.withhold_first_load) issue_load256<STAGES, kQdy>(s, &map_gate, &map_up, &map_gy, p, n, pol);
