@@ -45,6 +45,12 @@
  * different streams may run concurrently; concurrent calls must not share
  * output buffers.  Inputs and outputs must not overlap.
  *
+ * Stream order: the op's kernel is launched with programmatic stream
+ * serialization, so its blocks may start while the kernel before it on the
+ * stream is finishing; they read and write the arrays only after that
+ * kernel has completed.  Before that point a block only prefetches the first
+ * input tiles it will read into L2, which changes no value it reads.
+ *
  * Per-device state: the library sets up, once per device and process, the
  * kernels' attributes, the copy streams and events of sdq_fuse_host, and
  * the device address of sdq_fuse_host_noalloc's array.  All of it belongs

@@ -39,3 +39,17 @@ def test_algorithmic_bytes():
     w = W.BY_NAME["swiglu_bwd_int8_M4096_K1408"]
     assert w.algorithmic_bytes() == 52445184
     assert bench.int8_grad_y_bytes(w) == 52445184 - 4096 * 1408 + 4 * 4096 * 11
+
+
+def test_buffer_sets_rotate_at_least_three_and_exceed_three_l2():
+    """Consecutive timed calls never share buffers, and the sets together
+    exceed 3x L2 (no more sets than that needs, beyond the minimum of 3)."""
+    l2 = 126 * 2**20
+    assert bench.buffer_sets(1_067_974_656, l2) == 3   # one call larger than L2
+    for w in W.WORKLOADS:
+        per_call = w.algorithmic_bytes()
+        n = bench.buffer_sets(per_call, l2)
+        assert n >= 3
+        assert n * per_call >= 3 * l2
+        if n > 3:
+            assert (n - 1) * per_call < 3 * l2
