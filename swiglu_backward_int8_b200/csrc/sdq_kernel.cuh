@@ -25,7 +25,7 @@
 //   * each tile arrives as two 64-row stages; a stage is three TMA boxes
 //     (gate, up, grad_y; 64 x 128 bf16 each, 48 KB) in a STAGES-deep
 //     shared-memory ring.  Load n of a CTA is tile n/2, half n%2, so any thread
-//     can issue any load.  Each slot has an mbarrier (TMA byte count); the
+//     can issue any load.  A load completes on an mbarrier (TMA byte count); the
 //     warps release a slot through a shared counter and the warp that releases
 //     it last issues the load that goes next into it -- there is no producer
 //     warp, so every warp computes and may use 128 registers.
