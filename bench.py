@@ -80,6 +80,9 @@ def parse_args():
                     help="skip the per_workload list (every workload timed after the headline)")
     ap.add_argument("--per-workload-ms", type=float, default=50.0,
                     help="timed calls per workload: enough for about this many ms")
+    ap.add_argument("--per-call", type=int, default=50, metavar="N",
+                    help="per_workload entries also time N single calls, each after a write of "
+                         "2x L2, for their median / p10 / p90 (0: skip)")
     ap.add_argument("--traffic-probe", type=int, default=0, metavar="N",
                     help="no timing: N rounds of (read a 512 MB buffer, one call, read it again) "
                          "on one buffer set, for an ncu capture of the call's DRAM bytes including "
@@ -432,6 +435,38 @@ def measure_device(w: W.Workload, x_np, gy_np, steps: int, warmup: int, device, 
     return ms, (t0, t1), nsets
 
 
+def measure_per_call(w: W.Workload, x_np, gy_np, calls: int, device, warmup: int = 10) -> dict:
+    """Single calls, each after a write of 2x L2 (so it finds none of its data
+    in L2) and timed alone by CUDA events around it on the launching stream:
+    the latency of one cold call, launch included, as a median and p10/p90.
+    The graph-replayed figures time back-to-back calls instead."""
+    import torch
+    import swiglu_backward_int8_b200 as sdq
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    x = _to_device_bf16(x_np, device)
+    g = _to_device_bf16(gy_np, device)
+    outs = sdq.allocate_outputs(w.M, w.K, device, group_size=w.group_size)
+    stream = torch.cuda.current_stream(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(calls)]
+    for k in range(warmup + calls):
+        flush.fill_(k & 0xFF)
+        if k >= warmup:
+            evs[k - warmup][0].record(stream)
+        sdq.silu_dot_fwd_bwd_quant_fuse(x, g, *outs, w.group_size)
+        if k >= warmup:
+            evs[k - warmup][1].record(stream)
+    torch.cuda.synchronize(device)
+    st = sdq.sdq_device_status(stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError(f"device status {sdq.status_string(st)}")
+    us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
+    p10, p50, p90 = np.percentile(us, [10, 50, 90])
+    return {"median": float(p50), "p10": float(p10), "p90": float(p90), "calls": calls,
+            "l2_flush_bytes": 2 * l2}
+
+
 def measure_e2e(w: W.Workload, x_np, gy_np, steps: int, device):
     import torch
     import swiglu_backward_int8_b200 as sdq
@@ -520,11 +555,17 @@ def run_sdq(args):
             oms = parallel.max_over_ranks(oms, device)
             us = oms / osteps * 1e3
             gbs = ow.algorithmic_bytes() / (us * 1e-6) / 1e9
-            per.append({"workload": ow.name, "M": ow.M, "K": ow.K, "us_per_call": us,
-                        "GB_s": gbs, "frac_of_measured_hbm": gbs / peak, "frac_of_8TBs": gbs / 8000,
-                        "algorithmic_bytes_per_launch": ow.algorithmic_bytes(),
-                        "steps": osteps, "buffer_sets": ons,
-                        "clocks_sm_mhz": sampler.summary(o0, o1).get("sm_mhz")})
+            entry = {"workload": ow.name, "M": ow.M, "K": ow.K, "us_per_call": us,
+                     "GB_s": gbs, "frac_of_measured_hbm": gbs / peak, "frac_of_8TBs": gbs / 8000,
+                     "algorithmic_bytes_per_launch": ow.algorithmic_bytes(),
+                     "steps": osteps, "buffer_sets": ons,
+                     "clocks_sm_mhz": sampler.summary(o0, o1).get("sm_mhz")}
+            if args.per_call > 0:   # this rank's own device only: no collective
+                try:
+                    entry["per_call_us"] = measure_per_call(ow_r, ox, og, args.per_call, device)
+                except Exception as exc:   # a side measurement never costs the line
+                    entry["per_call_us"] = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+            per.append(entry)
             del ox, og
 
     per_fmt = None
@@ -590,6 +631,10 @@ def run_sdq(args):
         }
         if per is not None:
             line["per_workload"] = per
+            for e in per:   # per_workload runs the page's format at group size 128
+                if (e["workload"] == w.name and "per_call_us" in e and fmt == PAGE_FORMAT
+                        and w.group_size == 128):
+                    line["per_call_us"] = e["per_call_us"]
         if per_fmt is not None:
             line["per_format"] = per_fmt
         if with_y is not None:
